@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200: long-context prefill tokens/s and
+decode-step state GB/s, each against the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One "step" is one chunked prefill of the long-context workload (B=1, H=32,
+T=131072, d=128, bf16 q/k/v, fp32 gates, zero S0): the chunk-parallel kernel
+and the sequential carry kernel. The decode workload (256 sequences x 32 heads,
+128 x 128 fp32 state, bf16 q/k/v) is timed the same way and reported under
+"decode". Inputs are seeded synthetic tensors resident in HBM before the timed
+region; every workload's inputs are larger than the 126 MB L2, so no flush is
+needed between iterations. Under torchrun each rank runs its own independent
+problem (weak scaling, no collective on the data path) and the time is the max
+over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_132_b200 import inputs as I  # noqa: E402
+
+METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM peak, "
+          "1×B200")
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_setup(gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:  # noqa: BLE001 - clocks are best effort
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:  # noqa: BLE001
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags)
+                          if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def time_region(fn_step, steps, stream, marks=0):
+    """Run ``fn_step(i, events)`` for i < steps between two events on ``stream``.
+    ``marks`` extra events per step are handed to fn_step to bracket kernels.
+    Returns (total ms, [[ms between consecutive marks] per step])."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(marks)] for _ in range(steps)]
+    start.record(stream)
+    for i in range(steps):
+        fn_step(i, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(marks - 1)]
+           for i in range(steps)]
+    return start.elapsed_time(end), per
+
+
+# ----------------------------------------------------------------------------- our arm
+def bench_prefill(preset, steps, warmup, world, rank, dev, peaks, clocks=None):
+    from gated_delta_rule_132_b200 import kda
+    x = I.make_preset(preset, device=f"cuda:{dev}") if rank == 0 else \
+        I.make_prefill(preset.B, preset.T, preset.H, preset.d, preset.dtype, preset.gate_shift,
+                       preset.s0_std, preset.seed + 1000 * rank, device=f"cuda:{dev}")
+    call = kda.ChunkFwdCall(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"],
+                            x["cu_seqlens"], x["scale"])
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        call.run()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    def step(i, ev):
+        ev[0].record(stream)
+        call.prepare()
+        ev[1].record(stream)
+        call.carry()
+        ev[2].record(stream)
+
+    if clocks is not None:
+        with clocks:
+            total_ms, per = time_region(step, steps, stream, marks=3)
+    else:
+        total_ms, per = time_region(step, steps, stream, marks=3)
+    barrier(world)
+    ms = max_over_ranks(total_ms / steps, world)
+    prep_ms = statistics.mean(p[0] for p in per)
+    carry_ms = statistics.mean(p[1] for p in per)
+    tokens = x["q"].shape[0] * x["q"].shape[1]
+    token_heads = tokens * preset.H
+    d = preset.d
+    in_b = 3 * d * x["q"].element_size() + 4 * d + 4     # q,k,v + log_alpha + beta
+    out_b = d * x["q"].element_size()                     # o
+    n_seq = 1 if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
+    n_seq = preset.B if x["cu_seqlens"] is None else n_seq
+    state_b = n_seq * preset.H * d * d * 4 * (2 if x["S0"] is not None else 1)
+    op_bytes = token_heads * (in_b + out_b) + state_b
+    ws_bytes = call.workspace.numel()
+    return dict(x=x, call=call, ms=ms, prep_ms=prep_ms, carry_ms=carry_ms, tokens=tokens,
+                token_heads=token_heads, op_bytes=op_bytes, in_bytes=token_heads * in_b,
+                out_bytes=token_heads * out_b + state_b, ws_bytes=ws_bytes)
+
+
+def bench_decode(P, steps, warmup, world, rank, dev):
+    from gated_delta_rule_132_b200 import kda
+    devs = f"cuda:{dev}"
+    S = I.make_decode_state(P.N, P.H, P.d, P.s_std, P.seed + 1000 * rank, device=devs)
+    toks = [I.make_decode_token(P.N, P.H, P.d, P.dtype, P.gate_shift,
+                                seed=P.step_seed0 + i + 100000 * rank, device=devs)
+            for i in range(warmup + steps)]
+    o = torch.empty(P.N, P.H, P.d, dtype=P.dtype, device=devs)
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        kda.kda_decode_step(**toks[i], S=S, o=o)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    def step(i, ev):
+        ev[0].record(stream)
+        kda.kda_decode_step(**toks[warmup + i], S=S, o=o)
+        ev[1].record(stream)
+
+    total_ms, per = time_region(step, steps, stream, marks=2)
+    barrier(world)
+    ms = max_over_ranks(total_ms / steps, world)
+    kern_ms = statistics.mean(p[0] for p in per)
+    units = P.N * P.H
+    state_b = 2 * units * P.d * P.d * 4
+    io_b = units * (3 * P.d * 2 + 4 * P.d + 4 + P.d * 2)
+    return dict(ms=ms, kern_ms=kern_ms, bytes=state_b + io_b, state_bytes=state_b)
+
+
+def bench_e2e(pre, steps, stream):
+    """The same prefill through the public call with host buffers: pinned host
+    inputs copied in, kda_chunk_fwd, o and S_final copied out, every step."""
+    from gated_delta_rule_132_b200 import kda
+    x, call = pre["x"], pre["call"]
+    names = ["q", "k", "v", "log_alpha", "beta"]
+    host = {n: x[n].cpu().pin_memory() for n in names}
+    dev = {n: x[n] for n in names}
+    o_h = torch.empty(call.o.shape, dtype=call.o.dtype, pin_memory=True)
+    s_h = torch.empty(call.S_final.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * 4
+
+    def one():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        kda.kda_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                          x["S0"], x["cu_seqlens"], x["scale"], o=call.o,
+                          S_final=call.S_final, workspace=call.workspace)
+        o_h.copy_(call.o, non_blocking=True)
+        s_h.copy_(call.S_final, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    total_ms, _ = time_region(lambda i, ev: one(), steps, stream)
+    return dict(ms=total_ms / steps, h2d=h2d, d2h=d2h)
+
+
+def cpu_baseline(pre_x, preset, budget_s=12.0):
+    """The fp64 oracle as it stands on this host's cores, on the first tokens of
+    the same workload (all heads), sized to roughly ``budget_s`` seconds."""
+    import oracle
+    cores = oracle.num_threads(0)
+    xs = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in pre_x.items()}
+
+    def run(T):
+        sl = lambda t: t[:, :T]
+        t0 = time.perf_counter()
+        oracle.forward(sl(xs["q"]), sl(xs["k"]), sl(xs["v"]), sl(xs["log_alpha"]),
+                       sl(xs["beta"]), xs["S0"], None, xs["scale"], n_threads=0)
+        return time.perf_counter() - t0
+
+    T = 256
+    dt = run(T)
+    T = int(min(preset.T, max(256, T * budget_s / max(dt, 1e-3))))
+    T = max(64, T // 64 * 64)
+    dt = run(T)
+    used = min(cores, preset.H * xs["q"].shape[0])
+    return {"value": T * xs["q"].shape[0] / dt, "unit": "tokens/s", "cores": used,
+            "kind": "oracle",
+            "sample": f"first {T} tokens x {preset.H} heads of the workload "
+                      f"({dt:.1f} s, fp64 token-by-token, {used} threads)"}
+
+
+def run_ours(args, world, rank, dev):
+    from gated_delta_rule_132_b200 import kda
+    kda.lib()
+    peaks, peak_kind = load_peaks()
+    preset = I.LONG
+    clocks = ClockSampler(dev)
+    pre = bench_prefill(preset, args.steps, args.warmup, world, rank, dev, peaks, clocks)
+    dec = bench_decode(I.DECODE, args.steps, args.warmup, world, rank, dev)
+    hbm = peaks["hbm_gbs"]
+    value = pre["tokens"] * world / (pre["ms"] / 1e3)
+
+    # Dominant prefill kernel and its roofline (HBM: bytes it must move / its time).
+    ws_per_launch = pre["ws_bytes"]
+    prep_bytes = pre["in_bytes"] + ws_per_launch
+    carry_bytes = ws_per_launch + pre["out_bytes"]
+    kernels = {
+        "prepare": {"ms": pre["prep_ms"], "bytes": prep_bytes},
+        "carry": {"ms": pre["carry_ms"], "bytes": carry_bytes},
+    }
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    ach = kernels[dom]["bytes"] / (kernels[dom]["ms"] / 1e3) / 1e9
+    roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": None,
+            "peak_source": peak_kind,
+            "bytes_per_launch": kernels[dom]["bytes"], "ms_per_launch": kernels[dom]["ms"]}
+    op_ach = pre["op_bytes"] / (pre["ms"] / 1e3) / 1e9
+    dec_ach = dec["bytes"] / (dec["kern_ms"] / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["ms"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; q,k L2-normalised, beta=sigmoid(N), "
+                "log_alpha=-softplus(N-3))",
+        "config": {"workload": preset.name, "B": preset.B, "T": preset.T, "H": preset.H,
+                   "d_k": preset.d, "d_v": preset.d, "chunk": 64,
+                   "l2": "inputs larger than L2 (no flush needed)",
+                   "parallelism": f"independent problem per GPU x{world}"},
+        "roofline": roof,
+        "op_roofline": {"bound": "hbm", "achieved": round(op_ach, 1), "peak": hbm,
+                        "unit": "GB/s", "frac": round(op_ach / hbm, 4),
+                        "bytes_per_step": pre["op_bytes"],
+                        "note": "algorithmic bytes of the whole prefill (q,k,v,log_alpha,"
+                                "beta in, o out, states) / step time"},
+        "kernels_ms": {n: round(v["ms"], 4) for n, v in kernels.items()},
+        "decode": {"workload": I.DECODE.name, "value": round(dec_ach, 1), "unit": "GB/s",
+                   "ms_per_step": round(dec["kern_ms"], 4),
+                   "roofline": {"kernel": "decode", "bound": "hbm",
+                                "achieved": round(dec_ach, 1), "peak": hbm, "unit": "GB/s",
+                                "frac": round(dec_ach / hbm, 4), "traffic": None,
+                                "bytes_per_launch": dec["bytes"]}},
+        "gpu_launches": 3 * args.steps,
+    }
+    c = clocks.summary()
+    line["clocks"] = c
+    if not args.no_e2e:
+        e = bench_e2e(pre, max(1, min(args.steps, args.e2e_steps)),
+                      torch.cuda.current_stream())
+        e_ms = max_over_ranks(e["ms"], world)
+        line["e2e"] = {"value": round(pre["tokens"] * world / (e_ms / 1e3), 1),
+                       "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
+                       "d2h_bytes_per_step": e["d2h"], "ms_per_step": round(e_ms, 3)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(pre["x"], preset)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    """The fp64 oracle as the reference implementation, on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    preset = I.LONG
+    T_s = args.ref_tokens
+    x = I.make_prefill(1, T_s, preset.H, preset.d, preset.dtype, preset.gate_shift, 0.0,
+                       preset.seed, device="cpu")
+    cores = oracle.num_threads(0)
+
+    def step():
+        oracle.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, None,
+                       x["scale"], n_threads=0)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = T_s / dt
+    used = min(cores, preset.H)
+    sample = (f"first {T_s} tokens x {preset.H} heads of {preset.name} per step "
+              f"(fp64 token-by-token, {used} threads)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": preset.name, "B": preset.B, "T": preset.T, "H": preset.H,
+                   "d_k": preset.d, "d_v": preset.d},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": used,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=1024,
+                    help="tokens per reference-arm step (all 32 heads)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, dev = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, dev)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+// kda_api.cu — the exported C ABI: argument checks, workspace sizing, dispatch.
+//
+// Every check here runs on the host before any launch and touches no device
+// state, so a rejected call has no side effects (and can be made without a GPU).
+#include <math.h>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_ok(int dk, int dv) { return dk == dv && (dk == 32 || dk == 64 || dk == 128); }
+bool dtype_ok(kda_dtype_t t) { return t == KDA_DTYPE_F32 || t == KDA_DTYPE_BF16; }
+
+// Shapes -> Problem (pointers left null); returns KDA_OK or the first problem found.
+kda_status_t describe(int B, int T, int H, int dk, int dv, int n_seqs, bool varlen,
+                      kda_dtype_t dt, kda::Problem *p)
+{
+    if (B < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return KDA_ERR_UNSUPPORTED;
+    if (!head_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (H > 65535) return KDA_ERR_UNSUPPORTED;
+    if (varlen && (B != 1 || n_seqs < 1)) return KDA_ERR_INVALID_ARG;
+    const long long total = (long long)B * T;
+    if (total > (long long)INT32_MAX - kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    const int N = varlen ? n_seqs : B;
+    long long chunks = varlen ? total / kda::kChunk + N
+                              : (long long)B * ((T + kda::kChunk - 1) / kda::kChunk);
+    if (chunks > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    *p = kda::Problem{};
+    p->N = N; p->B = B; p->T = T; p->H = H; p->dk = dk; p->dv = dv; p->dtype = dt;
+    p->total_tokens = total;
+    p->max_chunks = (int)chunks;
+    return KDA_OK;
+}
+
+bool use_tc(const kda::Problem &p, int algo) {
+    if (algo == KDA_ALGO_SIMT) return false;
+    return kda::tc_supported(p);
+}
+
+size_t required_bytes(const kda::Problem &p, bool tc) {
+    return tc ? kda::tc_workspace_layout(p).total : kda::simt_workspace_layout(p).total;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status_t s)
+{
+    switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARG: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported size or dtype";
+    case KDA_ERR_ALIGNMENT: return "buffer not 16-byte aligned";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+    case KDA_ERR_CUDA: return "CUDA error";
+    case KDA_ERR_DEVICE_STATUS: return "device reported an out-of-domain input";
+    }
+    return "unknown status";
+}
+
+int kda_version(void) { return 100; }
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                    kda_dtype_t dt)
+{
+    kda::Problem p;
+    const bool varlen = n_seqs > 0 && B == 1;
+    if (describe(B, T, H, dk, dv, n_seqs, varlen, dt, &p) != KDA_OK) return 0;
+    // Enough for whichever path kda_chunk_fwd selects (and for the SIMT path).
+    size_t s = required_bytes(p, false);
+    if (kda::tc_supported(p)) {
+        const size_t t = required_bytes(p, true);
+        if (t > s) s = t;
+    }
+    return s;
+}
+
+}  // extern "C"
+
+static kda_status_t chunk_fwd_phases(const void *q, const void *k, const void *v,
+                                     kda_dtype_t dt, const float *log_alpha,
+                                     const float *beta, const float *S0,
+                                     const int32_t *cu_seqlens, int n_seqs, int B, int T,
+                                     int H, int dk, int dv, float scale, void *o,
+                                     float *S_final, void *workspace, size_t workspace_bytes,
+                                     int algo, int phases, void *stream)
+{
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TCGEN05)
+        return KDA_ERR_INVALID_ARG;
+    kda::Problem p;
+    kda_status_t st = describe(B, T, H, dk, dv, n_seqs, cu_seqlens != nullptr, dt, &p);
+    if (st != KDA_OK) return st;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if (p.total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o))
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, o, S_final, workspace};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_ALIGNMENT;
+    const bool tc = use_tc(p, algo);
+    if (algo == KDA_ALGO_TCGEN05 && !tc) return KDA_ERR_UNSUPPORTED;
+    const size_t need = required_bytes(p, tc);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+
+    p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.S0 = S0;
+    p.cu_seqlens = cu_seqlens; p.scale = scale; p.o = o; p.S_final = S_final;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = tc ? kda::launch_tc_prefill(p, workspace, phases, s)
+                             : kda::launch_simt_prefill(p, workspace, phases, s);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" {
+
+#define KDA_CHUNK_ARGS q, k, v, dt, log_alpha, beta, S0, cu_seqlens, n_seqs, B, T, H, dk, dv, \
+    scale, o, S_final, workspace, workspace_bytes
+
+kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                              const float *log_alpha, const float *beta, const float *S0,
+                              const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                              int dk, int dv, float scale, void *o, float *S_final,
+                              void *workspace, size_t workspace_bytes, int algo, void *stream)
+{
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseAll, stream);
+}
+
+kda_status_t kda_chunk_fwd_prepare(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                                   const float *log_alpha, const float *beta, const float *S0,
+                                   const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                                   int dk, int dv, float scale, void *o, float *S_final,
+                                   void *workspace, size_t workspace_bytes, int algo,
+                                   void *stream)
+{
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhasePrepare, stream);
+}
+
+kda_status_t kda_chunk_fwd_carry(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                                 int dk, int dv, float scale, void *o, float *S_final,
+                                 void *workspace, size_t workspace_bytes, int algo, void *stream)
+{
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseCarry, stream);
+}
+
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                           const float *log_alpha, const float *beta, const float *S0,
+                           const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                           int dk, int dv, float scale, void *o, float *S_final,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    return kda_chunk_fwd_ex(q, k, v, dt, log_alpha, beta, S0, cu_seqlens, n_seqs, B, T, H,
+                            dk, dv, scale, o, S_final, workspace, workspace_bytes,
+                            KDA_ALGO_AUTO, stream);
+}
+
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                             const float *log_alpha, const float *beta, float *S, int N,
+                             int H, int dk, int dv, float scale, void *o, void *stream)
+{
+    if (N < 1 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || !head_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
+    const cudaError_t e = kda::launch_decode(q, k, v, dt, log_alpha, beta, S, N, H, dk, dv,
+                                             scale, o, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

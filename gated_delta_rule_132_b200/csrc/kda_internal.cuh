@@ -1,0 +1,74 @@
+// kda_internal.cuh — declarations shared by the library's translation units.
+// Nothing here is part of the public C ABI (include/kda.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// Chunk length of the chunked prefill (tokens per chunk).
+constexpr int kChunk = 64;
+// Width of the value-column slice one sequential-carry CTA owns on the SIMT path.
+constexpr int kSimtSlice = 32;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Problem description after host-side validation.
+struct Problem {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    const int32_t *cu_seqlens;  // device, or null (uniform sequences of length T)
+    int N;                      // number of sequences
+    int B, T, H, dk, dv;
+    float scale;
+    void *o;
+    float *S_final;
+    kda_dtype_t dtype;
+    long long total_tokens;     // B * T (packed time axis length)
+    int max_chunks;             // upper bound on chunks over all sequences
+};
+
+// Sequence plan in the workspace: for n in [0, N], the sanitised packed start
+// token seq_start[n] and first global chunk chunk_off[n] (both int32; entry N
+// holds the totals).
+struct Plan {
+    int32_t *seq_start;
+    int32_t *chunk_off;
+};
+
+// Byte layout of one prefill workspace.
+struct WorkspaceLayout {
+    size_t plan_bytes;      // seq_start + chunk_off
+    size_t chunk_bytes;     // per-chunk intermediates, all heads
+    size_t total;
+};
+
+WorkspaceLayout simt_workspace_layout(const Problem &p);
+WorkspaceLayout tc_workspace_layout(const Problem &p);
+
+cudaError_t launch_plan(const Problem &p, Plan plan, cudaStream_t stream);
+cudaError_t launch_decode(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                          const float *log_alpha, const float *beta, float *S, int N, int H,
+                          int dk, int dv, float scale, void *o, cudaStream_t stream);
+// Prefill phases: bit 0 = prepare (plan + chunk-parallel kernel), bit 1 = carry.
+enum : int { kPhasePrepare = 1, kPhaseCarry = 2, kPhaseAll = 3 };
+cudaError_t launch_simt_prefill(const Problem &p, void *workspace, int phases,
+                                cudaStream_t stream);
+cudaError_t launch_tc_prefill(const Problem &p, void *workspace, int phases,
+                              cudaStream_t stream);
+bool tc_supported(const Problem &p);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace kda

@@ -1,0 +1,219 @@
+"""Thin ctypes binding of the KDA C ABI (include/kda.h) for torch CUDA tensors.
+
+Argument marshalling only: these functions check dtypes/shapes, allocate the
+outputs and the workspace with torch (device memory is torch's job here), and
+pass raw pointers plus ``torch.cuda.current_stream()`` to the C entry points of
+the same names. Every step of the computation runs in the library's kernels;
+there is no fallback of any kind. If the library is missing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
+
+KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
+ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2}
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+          3: "KDA_ERR_ALIGNMENT", 4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA",
+          6: "KDA_ERR_DEVICE_STATUS"}
+
+_lib = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_f = ctypes.c_float
+
+
+class KdaError(RuntimeError):
+    """A KDA C entry point returned a non-OK status."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = lib().kda_status_string(status).decode()
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({msg})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libkda_b200.so``; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m gated_delta_rule_132_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_status_string.argtypes = [_i]
+        L.kda_version.restype = _i
+        L.kda_version.argtypes = []
+        L.kda_chunk_fwd_workspace_size.restype = _sz
+        L.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
+        common = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
+                  _vp, _vp, _vp, _sz]
+        L.kda_chunk_fwd.restype = _i
+        L.kda_chunk_fwd.argtypes = common + [_vp]
+        for fn in ("kda_chunk_fwd_ex", "kda_chunk_fwd_prepare", "kda_chunk_fwd_carry"):
+            getattr(L, fn).restype = _i
+            getattr(L, fn).argtypes = common + [_i, _vp]
+        L.kda_decode_step.restype = _i
+        L.kda_decode_step.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _f,
+                                      _vp, _vp]
+        _lib = L
+    return _lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"q/k/v must be bf16 or fp32, got {t.dtype}")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs=0, dtype=torch.bfloat16) -> int:
+    """Bytes of workspace :func:`kda_chunk_fwd` needs (C: same name)."""
+    d = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(lib().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs, d))
+
+
+class ChunkFwdCall:
+    """One prefill problem marshalled for the C ABI: the checked tensors, the
+    outputs, the workspace and the ctypes argument list. Calling ``run``,
+    ``prepare`` or ``carry`` enqueues ``kda_chunk_fwd_ex`` or one of its two
+    phases on ``stream`` (default: the current torch stream)."""
+
+    def __init__(self, q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None,
+                 output_final_state=True, workspace=None, o=None, S_final=None,
+                 algo="auto"):
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        dtype = q.dtype
+        _dt(q)
+        for t, name in ((q, "q"), (k, "k")):
+            _need(t, name, dtype, (B, T, H, dk))
+        _need(v, "v", dtype, (B, T, H, dv))
+        _need(log_alpha, "log_alpha", torch.float32, (B, T, H, dk))
+        _need(beta, "beta", torch.float32, (B, T, H))
+        if cu_seqlens is not None:
+            _need(cu_seqlens, "cu_seqlens", torch.int32)
+            N = cu_seqlens.shape[0] - 1
+        else:
+            N = B
+        if S0 is not None:
+            _need(S0, "S0", torch.float32, (N, H, dk, dv))
+        if scale is None:
+            scale = dk ** -0.5
+        if o is None:
+            o = torch.empty((B, T, H, dv), dtype=dtype, device=q.device)
+        else:
+            _need(o, "o", dtype, (B, T, H, dv))
+        if output_final_state and S_final is None:
+            S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+        elif S_final is not None:
+            _need(S_final, "S_final", torch.float32, (N, H, dk, dv))
+        n_seqs = N if cu_seqlens is not None else 0
+        need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs, dtype)
+        if workspace is None:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        self.tensors = (q, k, v, log_alpha, beta, S0, cu_seqlens, workspace)
+        self.o, self.S_final, self.workspace = o, S_final, workspace
+        self.args = [_p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S0),
+                     _p(cu_seqlens), int(n_seqs), B, T, H, dk, dv, float(scale), _p(o),
+                     _p(S_final), _p(workspace), workspace.numel() * workspace.element_size(),
+                     ALGOS[algo]]
+
+    def _call(self, fn, stream):
+        st = getattr(lib(), fn)(*self.args, _stream(stream))
+        if st != 0:
+            raise KdaError(fn, st)
+        return self.o, self.S_final
+
+    def run(self, stream=None):
+        return self._call("kda_chunk_fwd_ex", stream)
+
+    def prepare(self, stream=None):
+        return self._call("kda_chunk_fwd_prepare", stream)
+
+    def carry(self, stream=None):
+        return self._call("kda_chunk_fwd_carry", stream)
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None,
+                  output_final_state=True, workspace=None, o=None, S_final=None,
+                  algo="auto", stream=None):
+    """Chunked KDA prefill (C: ``kda_chunk_fwd`` / ``kda_chunk_fwd_ex``).
+
+    q, k [B,T,H,dk] and v [B,T,H,dv] in bf16 or fp32; log_alpha [B,T,H,dk] fp32;
+    beta [B,T,H] fp32; S0 [N,H,dk,dv] fp32 or None; cu_seqlens int32 [N+1] or None
+    (then N = B). Returns (o [B,T,H,dv] in q's dtype, S_final [N,H,dk,dv] fp32 or None).
+    """
+    return ChunkFwdCall(q, k, v, log_alpha, beta, S0, cu_seqlens, scale, output_final_state,
+                        workspace, o, S_final, algo).run(stream)
+
+
+def kda_chunk_fwd_prepare(*args, stream=None, **kwargs) -> ChunkFwdCall:
+    """The chunk-parallel phase (C: ``kda_chunk_fwd_prepare``). Takes the
+    arguments of :func:`kda_chunk_fwd` and returns the marshalled call, whose
+    ``carry()`` runs the sequential phase on the same workspace."""
+    call = ChunkFwdCall(*args, **kwargs)
+    call.prepare(stream)
+    return call
+
+
+def kda_chunk_fwd_carry(call: ChunkFwdCall, stream=None):
+    """The sequential phase (C: ``kda_chunk_fwd_carry``) of a prepared call."""
+    return call.carry(stream)
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None):
+    """One recurrent decode step (C: ``kda_decode_step``); updates S in place.
+
+    q, k [N,H,dk]; v [N,H,dv] (bf16 or fp32); log_alpha [N,H,dk] fp32; beta [N,H]
+    fp32; S [N,H,dk,dv] fp32. Returns o [N,H,dv] in q's dtype.
+    """
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dtype = q.dtype
+    _dt(q)
+    _need(q, "q", dtype, (N, H, dk))
+    _need(k, "k", dtype, (N, H, dk))
+    _need(v, "v", dtype, (N, H, dv))
+    _need(log_alpha, "log_alpha", torch.float32, (N, H, dk))
+    _need(beta, "beta", torch.float32, (N, H))
+    _need(S, "S", torch.float32, (N, H, dk, dv))
+    if scale is None:
+        scale = dk ** -0.5
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=dtype, device=q.device)
+    else:
+        _need(o, "o", dtype, (N, H, dv))
+    st = lib().kda_decode_step(_p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S),
+                               N, H, dk, dv, float(scale), _p(o), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_decode_step", st)
+    return o

@@ -1,0 +1,168 @@
+/*
+ * kda.h — C ABI of the KDA (Kimi Delta Attention) library for NVIDIA B200 (sm_100a).
+ *
+ * The operation. "Kimi Linear：让长上下文大模型真正实用的线性注意力架构" (juejin.cn),
+ * section 三 5️⃣ gives the KDA update rule
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *
+ * (beta = learning rate, alpha = forget rate, S = memory state); section 三 1️⃣
+ * says the forget rate is per channel (alpha_t[i], one per key channel). The
+ * library reads out with the updated state, o_t = scale * S_t^T q_t, and takes
+ * the gate in log space, alpha_t = exp(log_alpha_t). S is dk x dv per head, so
+ * Diag(alpha_t) scales the dk rows of S.
+ *
+ * Layouts. Every tensor is a dense, row-major DEVICE buffer, 16-byte aligned:
+ *   q, k        [B, T, H, dk]   dtype given by qkv_dtype (fp32 or bf16)
+ *   v, o        [B, T, H, dv]   qkv_dtype (o has the same dtype as q, k, v)
+ *   log_alpha   [B, T, H, dk]   fp32, expected <= 0 (alpha in (0, 1])
+ *   beta        [B, T, H]       fp32
+ *   S0, S_final [N, H, dk, dv]  fp32, dv contiguous
+ * Sequences: without cu_seqlens, N = B and row b of the batch is one sequence of
+ * T tokens. With cu_seqlens (int32 [n_seqs + 1], device memory, cu_seqlens[0] = 0,
+ * non-decreasing, cu_seqlens[n_seqs] = T) the batch must have B = 1 and sequence
+ * n owns the packed tokens [cu_seqlens[n], cu_seqlens[n+1]); N = n_seqs. Zero-
+ * length sequences are allowed (their S_final equals their S0).
+ *
+ * Supported sizes: dk = dv in {32, 64, 128}. bf16 inputs with dk = dv = 128 run on
+ * the tcgen05 tensor-core path; all other supported cases run on the fp32 SIMT
+ * path (see kda_chunk_fwd_ex).
+ *
+ * Ownership and asynchrony. The caller owns every buffer, including the
+ * workspace; the library allocates no device memory and never synchronises the
+ * stream. Calls are enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ * the legacy default stream) and return once the launches are queued. Buffers
+ * must stay valid until the stream reaches that point. Concurrent calls on
+ * different streams need separate workspaces.
+ *
+ * Errors. Arguments are checked on the host before anything is launched; a bad
+ * argument returns an error status and launches nothing. A failed launch returns
+ * KDA_ERR_CUDA. The library never aborts, exits or traps.
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad cu_seqlens shape */
+    KDA_ERR_UNSUPPORTED = 2,   /* head size or dtype the library does not implement */
+    KDA_ERR_ALIGNMENT = 3,     /* a buffer is not 16-byte aligned */
+    KDA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    KDA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    KDA_ERR_DEVICE_STATUS = 6  /* the device reported an out-of-domain input */
+} kda_status_t;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype_t;
+
+/* Prefill algorithm selector for kda_chunk_fwd_ex. */
+typedef enum {
+    KDA_ALGO_AUTO = 0,    /* tcgen05 path when supported, else SIMT */
+    KDA_ALGO_SIMT = 1,    /* fp32 CUDA-core path: any supported dtype and size */
+    KDA_ALGO_TCGEN05 = 2  /* tensor-core path: bf16, dk = dv = 128 only */
+} kda_algo_t;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *kda_status_string(kda_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int kda_version(void);
+
+/*
+ * Workspace bytes that kda_chunk_fwd needs for this problem (0 on invalid
+ * sizes). The workspace holds the per-chunk intermediate matrices of the
+ * chunked form between the chunk-parallel and the sequential kernel; it is
+ * device memory owned by the caller, needs no initialisation and may be reused
+ * across calls on the same stream. For varlen calls pass B = 1, T = total
+ * packed tokens and n_seqs = number of sequences; otherwise n_seqs is ignored.
+ */
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                    kda_dtype_t qkv_dtype);
+
+/*
+ * Chunked prefill: runs the recurrence over every sequence from S0 (NULL = zero
+ * state), writes o for every token and, if S_final is not NULL, the state after
+ * each sequence's last token. Source: the update rule above ("Kimi Linear"
+ * juejin.cn page, section 三 5️⃣), evaluated in the exact chunked form (64-token
+ * chunks, a triangular solve per chunk, fp32 state carried on chip between
+ * chunks); results equal the token-by-token recurrence up to rounding.
+ *
+ *   q, k, v, o       qkv_dtype device buffers (layouts above)
+ *   log_alpha, beta  fp32 device buffers
+ *   S0, S_final      fp32 [N, H, dk, dv] or NULL; S0 and S_final may alias
+ *   cu_seqlens       int32 device buffer [n_seqs + 1] or NULL (then n_seqs is ignored)
+ *   scale            read-out scale (commonly dk^-0.5)
+ *   workspace        >= kda_chunk_fwd_workspace_size(...) bytes of device memory
+ *   stream           cudaStream_t or NULL
+ * T = 0 is allowed and only copies S0 to S_final (zeros without S0).
+ */
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                           const float *log_alpha, const float *beta, const float *S0,
+                           const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                           int dk, int dv, float scale, void *o, float *S_final,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* kda_chunk_fwd with an explicit algorithm choice (kda_algo_t). Asking for
+ * KDA_ALGO_TCGEN05 on a problem it does not support returns KDA_ERR_UNSUPPORTED. */
+kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                              const float *log_alpha, const float *beta, const float *S0,
+                              const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                              int dk, int dv, float scale, void *o, float *S_final,
+                              void *workspace, size_t workspace_bytes, int algo,
+                              void *stream);
+
+/*
+ * The two phases of kda_chunk_fwd_ex, exported separately (same arguments, same
+ * workspace). kda_chunk_fwd_ex(...) is exactly kda_chunk_fwd_prepare(...)
+ * followed by kda_chunk_fwd_carry(...) on the same stream.
+ *   prepare: the chunk-parallel phase. Plans the sequences and, for every
+ *            64-token chunk and head, forms the gate cumulative sums, the
+ *            intra-chunk matrices and the triangular solve, storing the chunk's
+ *            intermediates in the workspace. Reads q, k, v, log_alpha, beta.
+ *   carry:   the sequential phase. Walks each sequence's chunks in order with
+ *            the fp32 state on chip, writing o and S_final. Reads the workspace,
+ *            S0 and cu_seqlens-derived plan; does not read q, k, v or the gates.
+ * Useful to time the phases or to run the chunk-parallel phase ahead of time.
+ */
+kda_status_t kda_chunk_fwd_prepare(const void *q, const void *k, const void *v,
+                                   kda_dtype_t qkv_dtype, const float *log_alpha,
+                                   const float *beta, const float *S0,
+                                   const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                                   int dk, int dv, float scale, void *o, float *S_final,
+                                   void *workspace, size_t workspace_bytes, int algo,
+                                   void *stream);
+kda_status_t kda_chunk_fwd_carry(const void *q, const void *k, const void *v,
+                                 kda_dtype_t qkv_dtype, const float *log_alpha,
+                                 const float *beta, const float *S0,
+                                 const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                                 int dk, int dv, float scale, void *o, float *S_final,
+                                 void *workspace, size_t workspace_bytes, int algo,
+                                 void *stream);
+
+/*
+ * Recurrent decode: one new token for each of N independent sequences. Applies
+ * the update rule once per (sequence, head) to the state S in place and writes
+ * o = scale * S_new^T q. Source: the same update rule; the kernel evaluates it
+ * in one pass over S using o = scale * (S'^T q + (k^T q) u) with
+ * S' = Diag(alpha) S and u = beta (v - S'^T k), so S is read once and written
+ * once.
+ *
+ *   q, k        qkv_dtype [N, H, dk]      v, o   qkv_dtype [N, H, dv]
+ *   log_alpha   fp32 [N, H, dk]           beta   fp32 [N, H]
+ *   S           fp32 [N, H, dk, dv], read and overwritten
+ */
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                             const float *log_alpha, const float *beta, float *S, int N,
+                             int H, int dk, int dv, float scale, void *o, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H */

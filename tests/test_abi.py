@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_132_b200 import build, kda
+    build.build()
+    return kda.lib()
+
+
+def declared_functions():
+    src = open(HEADER, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(kda_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+                     "kda_status_string"):
+        assert required in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_symbol_exported(L, name):
+    assert hasattr(L, name), f"{name} declared in include/kda.h but not exported"
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.kda_status_string(s)
+    assert L.kda_version() >= 100
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def _chunk(L, **kw):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), dt=1, la=_fake(), beta=_fake(), S0=None,
+             cu=None, n_seqs=0, B=1, T=64, H=2, dk=128, dv=128, scale=0.1, o=_fake(),
+             Sf=None, ws=_fake(), ws_bytes=1 << 40, algo=0, stream=None)
+    a.update(kw)
+    return L.kda_chunk_fwd_ex(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["S0"],
+                              a["cu"], a["n_seqs"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                              a["scale"], a["o"], a["Sf"], a["ws"], a["ws_bytes"], a["algo"],
+                              a["stream"])
+
+
+# Every case below must be rejected on the host: the fake device pointers are
+# never dereferenced and no CUDA call is made.
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(beta=None), 1), (dict(o=None), 1),
+    (dict(B=0), 1), (dict(T=-1), 1), (dict(H=0), 1),
+    (dict(dk=96, dv=96), 2), (dict(dk=128, dv=64), 2), (dict(dt=7), 2),
+    (dict(q=_fake(0x10004)), 3), (dict(la=_fake(0x10008)), 3), (dict(Sf=_fake(0x10001)), 3),
+    (dict(ws=None), 4), (dict(ws_bytes=16), 4),
+    (dict(cu=_fake(), n_seqs=0), 1), (dict(cu=_fake(), n_seqs=2, B=2), 1),
+    (dict(algo=9), 1), (dict(scale=float("nan")), 1),
+    (dict(dk=64, dv=64, algo=2), 2), (dict(dt=0, algo=2), 2),
+])
+def test_chunk_fwd_rejects(L, kw, status):
+    assert _chunk(L, **kw) == status
+
+
+def test_workspace_size(L):
+    a = L.kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 0, 1)
+    b = L.kda_chunk_fwd_workspace_size(4, 4097, 16, 128, 128, 0, 1)
+    assert 0 < a < b
+    assert L.kda_chunk_fwd_workspace_size(1, 1000, 4, 64, 64, 3, 0) > 0
+    assert L.kda_chunk_fwd_workspace_size(1, 100, 4, 96, 96, 0, 0) == 0
+    assert L.kda_chunk_fwd_workspace_size(0, 100, 4, 64, 64, 0, 0) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=0), 1), (dict(S=None), 1), (dict(dk=48, dv=48), 2), (dict(dt=3), 2),
+    (dict(S=_fake(0x10008)), 3), (dict(o=_fake(0x10002)), 3), (dict(scale=float("inf")), 1),
+])
+def test_decode_rejects(L, kw, status):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), dt=1, la=_fake(), beta=_fake(), S=_fake(),
+             N=4, H=2, dk=128, dv=128, scale=0.1, o=_fake(), stream=None)
+    a.update(kw)
+    assert L.kda_decode_step(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["S"],
+                             a["N"], a["H"], a["dk"], a["dv"], a["scale"], a["o"],
+                             a["stream"]) == status
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from gated_delta_rule_132_b200 import kda
+    monkeypatch.setattr(kda, "_lib", None)
+    monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        kda.lib()

@@ -1,0 +1,169 @@
+"""kda_chunk_fwd on the GPU against the fp64 oracle, on both prefill paths."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from common import TOL, rel_l2, to_cuda
+from gated_delta_rule_132_b200 import inputs as I
+from gated_delta_rule_132_b200 import kda
+
+pytestmark = pytest.mark.gpu
+
+# (algo, dtype, d) combinations each path implements.
+PATHS = [("simt", torch.float32, 32), ("simt", torch.float32, 64),
+         ("simt", torch.float32, 128), ("simt", torch.bfloat16, 64),
+         ("simt", torch.bfloat16, 128), ("tcgen05", torch.bfloat16, 128)]
+
+
+def _has_tc():
+    return kda.lib().kda_chunk_fwd_workspace_size(1, 64, 1, 128, 128, 0, 1) > 0
+
+
+def run_both(x, algo="auto", heads=None, output_final_state=True):
+    """GPU result and oracle result on the same inputs (optionally only some heads
+    go through the oracle)."""
+    g = to_cuda(x)
+    o, Sf = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["S0"],
+                              g["cu_seqlens"], x["scale"], output_final_state, algo=algo)
+    torch.cuda.synchronize()
+    sel = slice(None) if heads is None else heads
+    ref_in = {k: (x[k][:, :, sel] if x[k] is not None and k != "S0" and k != "cu_seqlens"
+                  else x[k]) for k in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens")}
+    if x["S0"] is not None:
+        ref_in["S0"] = x["S0"][:, sel]
+    o_ref, S_ref = oracle.forward(ref_in["q"], ref_in["k"], ref_in["v"], ref_in["log_alpha"],
+                                  ref_in["beta"], ref_in["S0"], ref_in["cu_seqlens"],
+                                  scale=x["scale"])
+    o_gpu = o[:, :, sel]
+    S_gpu = None if Sf is None else Sf[:, sel]
+    return o_gpu, S_gpu, o_ref, S_ref
+
+
+def _skip_unless(algo):
+    if algo == "tcgen05" and not _has_tc():
+        pytest.skip("tcgen05 path not built")
+
+
+def test_tiny_fp32_config():
+    """B=1, H=2, T=64, d=32, fp32: rel-L2 <= 1e-4 on o and S_final."""
+    x = I.make_preset(I.TINY)
+    o, Sf, o_ref, S_ref = run_both(x)
+    assert rel_l2(o, o_ref) <= 1e-4
+    assert rel_l2(Sf, S_ref) <= 1e-4
+
+
+@pytest.mark.parametrize("algo,dtype,d", PATHS)
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_lengths_and_tails(algo, dtype, d, T):
+    _skip_unless(algo)
+    x = I.make_prefill(2, T, 3, d, dtype, gate_shift=-1.0, s0_std=0.05, seed=T * 7 + d)
+    o, Sf, o_ref, S_ref = run_both(x, algo=algo)
+    assert rel_l2(o, o_ref) <= TOL[dtype]
+    assert rel_l2(Sf, S_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("algo,dtype,d", PATHS)
+def test_varlen_with_empty_and_ragged_sequences(algo, dtype, d):
+    _skip_unless(algo)
+    lengths = [1, 64, 0, 65, 127, 3, 190, 0, 64]
+    x = I.make_prefill(1, 0, 2, d, dtype, gate_shift=-1.0, s0_std=0.05, seed=31 + d,
+                       lengths=lengths)
+    o, Sf, o_ref, S_ref = run_both(x, algo=algo)
+    assert rel_l2(o, o_ref) <= TOL[dtype]
+    assert rel_l2(Sf, S_ref) <= TOL[dtype]
+    # zero-length sequences return their S0 exactly
+    assert torch.equal(Sf[2].cpu(), x["S0"][2]) and torch.equal(Sf[7].cpu(), x["S0"][7])
+
+
+@pytest.mark.parametrize("algo,dtype,d", PATHS)
+def test_zero_state_and_no_final_state(algo, dtype, d):
+    _skip_unless(algo)
+    x = I.make_prefill(1, 150, 2, d, dtype, gate_shift=0.0, s0_std=0.0, seed=5)
+    o, Sf, o_ref, S_ref = run_both(x, algo=algo, output_final_state=False)
+    assert Sf is None
+    assert rel_l2(o, o_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("algo", ["simt", "tcgen05"])
+def test_empty_time_axis_copies_state(algo):
+    _skip_unless(algo)
+    x = I.make_prefill(3, 0, 2, 128, torch.bfloat16, s0_std=0.05, seed=9)
+    g = to_cuda(x)
+    o, Sf = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["S0"],
+                              algo=algo)
+    assert o.numel() == 0 and torch.equal(Sf, g["S0"])
+    o, Sf = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None,
+                              algo=algo)
+    assert torch.count_nonzero(Sf) == 0
+
+
+@pytest.mark.parametrize("algo", ["simt", "tcgen05"])
+def test_split_prefill_equals_single_call(algo):
+    """forward(T) == forward(T1) then forward(T - T1) from its S_final (the state
+    is the whole checkpoint of a sequence)."""
+    _skip_unless(algo)
+    x = to_cuda(I.make_prefill(2, 300, 4, 128, torch.bfloat16, -1.0, 0.05, seed=12))
+    args = lambda s, e: (x["q"][:, s:e].contiguous(), x["k"][:, s:e].contiguous(),
+                         x["v"][:, s:e].contiguous(), x["log_alpha"][:, s:e].contiguous(),
+                         x["beta"][:, s:e].contiguous())
+    o, Sf = kda.kda_chunk_fwd(*args(0, 300), x["S0"], algo=algo)
+    oa, Sa = kda.kda_chunk_fwd(*args(0, 100), x["S0"], algo=algo)
+    ob, Sb = kda.kda_chunk_fwd(*args(100, 300), Sa, algo=algo)
+    assert rel_l2(torch.cat([oa, ob], 1), o.double().cpu().numpy()) <= 1e-2
+    assert rel_l2(Sb, Sf.double().cpu().numpy()) <= 1e-2
+
+
+@pytest.mark.parametrize("algo", ["simt", "tcgen05"])
+def test_deterministic_and_in_place_state(algo):
+    _skip_unless(algo)
+    x = to_cuda(I.make_prefill(2, 260, 4, 128, torch.bfloat16, -1.0, 0.05, seed=13))
+    a = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"])
+    o1, S1 = kda.kda_chunk_fwd(*a, x["S0"], algo=algo)
+    o2, S2 = kda.kda_chunk_fwd(*a, x["S0"], algo=algo)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    S = x["S0"].clone()
+    o3, S3 = kda.kda_chunk_fwd(*a, S, S_final=S, algo=algo)  # S0 aliases S_final
+    assert torch.equal(o3, o1) and torch.equal(S, S1)
+
+
+def test_chunked_config_full_size():
+    """B=4, H=16, T=4096, d=128, bf16, S0 ~ N(0, 0.01): every output checked."""
+    x = I.make_preset(I.CHUNKED)
+    o, Sf, o_ref, S_ref = run_both(x)
+    assert rel_l2(o, o_ref) <= 2e-2
+    assert rel_l2(Sf, S_ref) <= 2e-2
+
+
+@pytest.mark.slow
+def test_long_context_config_sampled_heads():
+    """B=1, H=32, T=131072, d=128, bf16, slow decay: the GPU runs all 32 heads;
+    the oracle checks 4 of them end to end (heads are independent)."""
+    x = I.make_preset(I.LONG)
+    heads = [0, 9, 21, 31]
+    o, Sf, o_ref, S_ref = run_both(x, heads=heads)
+    assert rel_l2(o, o_ref) <= 2e-2
+    assert rel_l2(Sf, S_ref) <= 2e-2
+
+
+@pytest.mark.slow
+def test_varlen_config_sampled_heads():
+    """8 packed sequences of seeded lengths in [1024, 65536], H=32, d=128, bf16,
+    per-sequence S0: the oracle checks every sequence on 3 heads."""
+    x = I.make_preset(I.VARLEN)
+    heads = [2, 17, 30]
+    o, Sf, o_ref, S_ref = run_both(x, heads=heads)
+    assert rel_l2(o, o_ref) <= 2e-2
+    assert rel_l2(Sf, S_ref) <= 2e-2
+
+
+@pytest.mark.parametrize("algo", ["simt", "tcgen05"])
+def test_prepare_then_carry_equals_one_call(algo):
+    _skip_unless(algo)
+    x = to_cuda(I.make_prefill(1, 0, 3, 128, torch.bfloat16, -1.0, 0.05, seed=14,
+                               lengths=[70, 1, 200]))
+    a = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], x["cu_seqlens"])
+    o1, S1 = kda.kda_chunk_fwd(*a, algo=algo)
+    call = kda.kda_chunk_fwd_prepare(*a, algo=algo)
+    o2, S2 = kda.kda_chunk_fwd_carry(call)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
