@@ -36,6 +36,9 @@ from gated_delta_rule_132_b200 import inputs as I  # noqa: E402
 
 METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM peak, "
           "1×B200")
+# Kernels one tcgen05 prefill call launches: plan, prep, exact fixup (exits at
+# once when no chunk needs it), carry. (The error-word reset is a memset.)
+LAUNCHES_PER_PREFILL = 4
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -148,11 +151,18 @@ def time_region(fn_step, steps, stream, marks=0):
 
 
 # ----------------------------------------------------------------------------- our arm
-def bench_prefill(preset, steps, warmup, world, rank, dev, peaks, clocks=None):
+def bench_prefill(preset, steps, warmup, world, rank, dev, peaks):
     from gated_delta_rule_132_b200 import kda
-    x = I.make_preset(preset, device=f"cuda:{dev}") if rank == 0 else \
-        I.make_prefill(preset.B, preset.T, preset.H, preset.d, preset.dtype, preset.gate_shift,
-                       preset.s0_std, preset.seed + 1000 * rank, device=f"cuda:{dev}")
+    if rank == 0:
+        x = I.make_preset(preset, device=f"cuda:{dev}")
+    else:  # an independent problem of the same shape on every other rank
+        lengths = None
+        if preset.n_varlen:
+            lengths = I.varlen_lengths(preset.n_varlen, preset.varlen_min, preset.varlen_max,
+                                       preset.seed)
+        x = I.make_prefill(preset.B, preset.T, preset.H, preset.d, preset.dtype,
+                           preset.gate_shift, preset.s0_std, preset.seed + 1000 * rank,
+                           lengths=lengths, device=f"cuda:{dev}")
     call = kda.ChunkFwdCall(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"],
                             x["cu_seqlens"], x["scale"])
     stream = torch.cuda.current_stream()
@@ -168,11 +178,7 @@ def bench_prefill(preset, steps, warmup, world, rank, dev, peaks, clocks=None):
         call.carry()
         ev[2].record(stream)
 
-    if clocks is not None:
-        with clocks:
-            total_ms, per = time_region(step, steps, stream, marks=3)
-    else:
-        total_ms, per = time_region(step, steps, stream, marks=3)
+    total_ms, per = time_region(step, steps, stream, marks=3)
     barrier(world)
     ms = max_over_ranks(total_ms / steps, world)
     prep_ms = statistics.mean(p[0] for p in per)
@@ -279,10 +285,12 @@ def run_ours(args, world, rank, dev):
     from gated_delta_rule_132_b200 import kda
     kda.lib()
     peaks, peak_kind = load_peaks()
-    preset = I.LONG
+    preset = {"long": I.LONG, "chunked": I.CHUNKED, "varlen": I.VARLEN}[args.workload]
     clocks = ClockSampler(dev)
-    pre = bench_prefill(preset, args.steps, args.warmup, world, rank, dev, peaks, clocks)
-    dec = bench_decode(I.DECODE, args.steps, args.warmup, world, rank, dev)
+    with clocks:
+        pre = bench_prefill(preset, args.steps, args.warmup, world, rank, dev, peaks)
+        dec = None if args.no_decode else bench_decode(I.DECODE, args.steps, args.warmup,
+                                                       world, rank, dev)
     hbm = peaks["hbm_gbs"]
     value = pre["tokens"] * world / (pre["ms"] / 1e3)
 
@@ -301,14 +309,13 @@ def run_ours(args, world, rank, dev):
             "peak_source": peak_kind,
             "bytes_per_launch": kernels[dom]["bytes"], "ms_per_launch": kernels[dom]["ms"]}
     op_ach = pre["op_bytes"] / (pre["ms"] / 1e3) / 1e9
-    dec_ach = dec["bytes"] / (dec["kern_ms"] / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["ms"], 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; q,k L2-normalised, beta=sigmoid(N), "
                 "log_alpha=-softplus(N-3))",
-        "config": {"workload": preset.name, "B": preset.B, "T": preset.T, "H": preset.H,
+        "config": {"workload": preset.name, "B": preset.B, "T": int(pre["tokens"]), "H": preset.H,
                    "d_k": preset.d, "d_v": preset.d, "chunk": 64,
                    "l2": "inputs larger than L2 (no flush needed)",
                    "parallelism": f"independent problem per GPU x{world}"},
@@ -319,14 +326,16 @@ def run_ours(args, world, rank, dev):
                         "note": "algorithmic bytes of the whole prefill (q,k,v,log_alpha,"
                                 "beta in, o out, states) / step time"},
         "kernels_ms": {n: round(v["ms"], 4) for n, v in kernels.items()},
-        "decode": {"workload": I.DECODE.name, "value": round(dec_ach, 1), "unit": "GB/s",
-                   "ms_per_step": round(dec["kern_ms"], 4),
-                   "roofline": {"kernel": "decode", "bound": "hbm",
-                                "achieved": round(dec_ach, 1), "peak": hbm, "unit": "GB/s",
-                                "frac": round(dec_ach / hbm, 4), "traffic": None,
-                                "bytes_per_launch": dec["bytes"]}},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": LAUNCHES_PER_PREFILL * args.steps,
     }
+    if dec is not None:
+        dec_ach = dec["bytes"] / (dec["kern_ms"] / 1e3) / 1e9
+        line["decode"] = {"workload": I.DECODE.name, "value": round(dec_ach, 1), "unit": "GB/s",
+                          "ms_per_step": round(dec["kern_ms"], 4),
+                          "roofline": {"kernel": "decode", "bound": "hbm",
+                                       "achieved": round(dec_ach, 1), "peak": hbm,
+                                       "unit": "GB/s", "frac": round(dec_ach / hbm, 4),
+                                       "traffic": None, "bytes_per_launch": dec["bytes"]}}
     c = clocks.summary()
     line["clocks"] = c
     if not args.no_e2e:
@@ -373,7 +382,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": preset.name, "B": preset.B, "T": preset.T, "H": preset.H,
+        "config": {"workload": preset.name, "B": preset.B, "T": int(pre["tokens"]), "H": preset.H,
                    "d_k": preset.d, "d_v": preset.d},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": used,
                          "kind": "oracle", "sample": sample},
@@ -389,6 +398,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["long", "chunked", "varlen"], default="long",
+                    help="prefill workload (default: the long-context one)")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -77,8 +77,10 @@ struct TcParams {
     __nv_bfloat16 *o;
     float *S_final;
     const int32_t *seq_start, *chunk_off;
-    uint8_t *rec;  // records
-    int *err;      // device error word
+    uint8_t *rec;      // records
+    int *err;          // device error word (pipeline timeouts)
+    int *fix_count;    // number of chunks listed for the exact fixup
+    int *fix_list;     // chunk * H + head, one per listed chunk
 };
 
 __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int c)
@@ -92,15 +94,17 @@ __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int c)
     return lo;
 }
 
-// ------------------------------------------------------------------- prep (v1)
-// fp32 CUDA-core prep: exact per-term gate exponents for A and P, forward
-// substitution for W and U~, then the record image.
+// ------------------------------------------------------------------- exact fixup
+// fp32 CUDA-core recomputation of one chunk's record with an exact exponential
+// for every gate difference in A and P and forward substitution for W and U~.
+// Used only for the chunks the tensor-core prep lists as outside the range of
+// its factorised exponentials (a decay of more than 80 nats inside half a
+// chunk); for ordinary gates the list is empty and the kernel exits at once.
 constexpr int kPrepThreads = 256;
 
-__global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(TcParams p)
+__device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
 {
     constexpr int DP = D + 1;
-    extern __shared__ float smem[];
     float *sk = smem;               // [C][DP]
     float *sq = sk + C * DP;        // [C][DP]
     float *sg = sq + C * DP;        // [C][DP]
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(TcParams p)
     float *sA = sv + C * D;         // [C][C+1]
     float *sb = sA + C * (C + 1);   // [C]
 
-    const int c = blockIdx.x, h = blockIdx.y, H = p.H;
+    const int H = p.H;
     const int n = find_seq(p.chunk_off, p.N, c);
     if (n < 0) return;
     const int t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
@@ -190,6 +194,467 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(TcParams p)
         a1[(kb + tc::sw128(r, 2 * (i & 63))) / 2] = __float2bfloat16_rn(sk[r * DP + i]);
         const int half = i >> 6, jj = i & 63;
         *reinterpret_cast<float *>(uu + half * 16384 + u_swz(r, jj)) = sv[r * D + i];
+    }
+    __syncthreads();  // the caller reuses shared memory for its next chunk
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams p)
+{
+    extern __shared__ float smem[];
+    const int count = *p.fix_count;
+    for (int idx = blockIdx.x; idx < count; idx += gridDim.x) {
+        const int e = p.fix_list[idx];
+        prep_exact_chunk(p, e / p.H, e % p.H, smem);
+    }
+}
+
+// ------------------------------------------------------------------- prep
+// Tensor-core prep. Per chunk and head (256 threads):
+//  1. Each thread owns 2 key channels x 16 tokens: loads q, k, v, log_alpha,
+//     forms the in-chunk cumulative log-decay g (quarter totals exchanged in
+//     shared memory), E_r = e^{g_r} and H_r = e^{g_C - g_r}, and writes Q~ and K^
+//     to the record and the MMA operands below to shared memory.
+//  2. The intra-chunk matrices A and P need e^{g_r - g_s} inside a contraction
+//     over channels, so it is split into a row factor and a column factor
+//     around a reference token: rows/cols of the first half use g_15, rows of
+//     the second half and every column against them use g_31. One MMA,
+//         D (128x96) = [K'_0; Q'_0; K'_1; Q'_1] (128x128) . [K''_0 | K''_1]^T,
+//     yields both diagonal 32x32 blocks and the off-diagonal 32x32 block of
+//     A (from k rows) and P (from q rows). Every factor is <= 1 except within a
+//     half, where it is bounded by the decay across at most 32 tokens; a chunk
+//     that would exceed e^80 there is listed for the exact fixup kernel.
+//  3. T = (I + A)^{-1} in fp32 by blocks of 16: the four diagonal blocks by
+//     substitution, then the off-diagonal blocks by distance,
+//     T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, as 16x16 products on all threads.
+//  4. [W | U~] = [T; 0] (128x64) . [beta K~ | beta V] (64x256) as one MMA; rows
+//     0..63 of the accumulator are the 64 tokens.
+//  5. Everything goes to the record in the carry kernel's operand layouts.
+constexpr int kPrep2Threads = 256;
+
+struct Prep2Smem {
+    static constexpr uint32_t kAop = 0;        // 32768: [kb][128 rows][128B]
+    static constexpr uint32_t kA = 0;          // fp32 A [64][65], after MMA-AP
+    static constexpr uint32_t kBop = 32768;    // 24576: [kb][96 rows][128B]
+    static constexpr uint32_t kT = 32768;      // fp32 T [64][65], after MMA-AP
+    static constexpr uint32_t kY = 49408;      // fp32 3 x [16][16] block products
+    static constexpr uint32_t kBK = 57344;     // 16384: (beta K~) MN-major image
+    static constexpr uint32_t kBV = 73728;     // 16384: (beta V) MN-major image (follows BK)
+    static constexpr uint32_t kTt = 90112;     // 16384: [T; 0], K-major rows r
+    // During step 1 the [T; 0] buffer is free: it holds the token-group totals
+    // and the per-channel constants (its zero rows are written after step 2).
+    static constexpr uint32_t kTot = kTt;          // 8192:  token-group totals [16][128]
+    static constexpr uint32_t kCst = kTt + 8192;   // 3584:  per-channel constants [7][128]
+    static constexpr uint32_t kB = 106496;     // 256:   beta [64]
+    static constexpr uint32_t kBar = 106752;   // barriers + tmem slot + flags
+    static constexpr uint32_t kBytes = kBar + 64 + 1024;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Y = sum_k A[ai + rr][aj + k] * T[tj0 + k][tc0 + cc] over k in [0,16), for the
+// thread's (rr, cc); matrices in the [64][65] fp32 layout.
+__device__ __forceinline__ float blk_dot(const float *A, int ar, int ac, const float *T, int tr,
+                                         int tc, int rr, int cc)
+{
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc += A[(ar + rr) * 65 + ac + k] * T[(tr + k) * 65 + tc + cc];
+    return acc;
+}
+
+__global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar_ap = reinterpret_cast<uint64_t *>(sm + Prep2Smem::kBar);
+    uint64_t *bar_wu = bar_ap + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ap + 2);
+    volatile int *abort = reinterpret_cast<volatile int *>(bar_ap + 3);
+    float *tot = reinterpret_cast<float *>(sm + Prep2Smem::kTot);    // [16][128] group totals
+    float *cst = reinterpret_cast<float *>(sm + Prep2Smem::kCst);    // [8][128] per channel
+    float *sbeta = reinterpret_cast<float *>(sm + Prep2Smem::kB);
+
+    const int c = blockIdx.x, h = blockIdx.y, H = p.H;
+    const int n = find_seq(p.chunk_off, p.N, c);
+    if (n < 0) return;  // uniform over the CTA: nothing allocated yet
+    const int t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
+    const int L = min(C, p.seq_start[n + 1] - t0);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    // 16-byte granules: channel octet `oc` (8 channels = one 16-byte swizzle
+    // chunk of a bf16 row) x token group `tg` (4 consecutive tokens)
+    const int oc = tid & 15, tg = tid >> 4;
+    const int c0 = 8 * oc;
+    const uint32_t kb = (uint32_t)(oc >> 3);   // K-block / MN atom
+    const uint32_t ck = (uint32_t)(oc & 7);    // chunk inside the 128-byte row
+
+    if (tid == 0) {
+        tc::mbar_init(bar_ap, 1);
+        tc::mbar_init(bar_wu, 1);
+        *abort = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) { tc::tmem_alloc(tmem_slot, 256); tc::tmem_relinquish(); }
+    if (tid < C) sbeta[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * H + h] : 0.f;
+
+    // ---- 1. loads and the cumulative log-decay
+    uint4 qv[4], kv[4], vv[4];
+    float g[4][8];
+    {
+        float run[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) run[j] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int r = tg * 4 + e;
+            uint4 q4 = make_uint4(0, 0, 0, 0), k4 = q4, v4 = q4;
+            float4 la0 = make_float4(0.f, 0.f, 0.f, 0.f), la1 = la0;
+            if (r < L) {
+                const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
+                q4 = __ldg(reinterpret_cast<const uint4 *>(p.q + off));
+                k4 = __ldg(reinterpret_cast<const uint4 *>(p.k + off));
+                v4 = __ldg(reinterpret_cast<const uint4 *>(p.v + off));
+                la0 = __ldg(reinterpret_cast<const float4 *>(p.log_alpha + off));
+                la1 = __ldg(reinterpret_cast<const float4 *>(p.log_alpha + off + 4));
+            }
+            qv[e] = q4; kv[e] = k4; vv[e] = v4;
+            run[0] += la0.x; run[1] += la0.y; run[2] += la0.z; run[3] += la0.w;
+            run[4] += la1.x; run[5] += la1.y; run[6] += la1.z; run[7] += la1.w;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) g[e][j] = run[j];
+        }
+        *reinterpret_cast<float4 *>(tot + tg * D + c0) = make_float4(run[0], run[1], run[2], run[3]);
+        *reinterpret_cast<float4 *>(tot + tg * D + c0 + 4) = make_float4(run[4], run[5], run[6], run[7]);
+    }
+    __syncthreads();
+    if (tid < D) {
+        // exclusive prefix over the 16 token groups of channel `tid`, plus the
+        // per-channel constants of the factorised exponentials
+        float run = 0.f, g15 = 0.f, g31 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (q == 4) g15 = run;
+            if (q == 8) g31 = run;
+            const float v = tot[q * D + tid];
+            tot[q * D + tid] = run;
+            run += v;
+        }
+        const float gC = run;
+        cst[0 * D + tid] = g15;
+        cst[1 * D + tid] = g31;
+        cst[2 * D + tid] = gC;
+        cst[3 * D + tid] = __expf(-g15);
+        cst[4 * D + tid] = __expf(-g31);
+        cst[5 * D + tid] = __expf(g15 - gC);
+        cst[6 * D + tid] = __expf(g31 - gC);
+        reinterpret_cast<float *>(p.rec + ((size_t)c * H + h) * Record::kBytes + Record::kG)[tid] =
+            __expf(gC);
+    }
+    // Multiplicative factors are exact while e^{g} cannot underflow; otherwise
+    // take every factor as a direct exponential of its difference.
+    const bool fast = __syncthreads_and(tid >= D || cst[2 * D + tid] > -80.f);
+
+    uint8_t *rec = p.rec + ((size_t)c * H + h) * Record::kBytes;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float go = tot[tg * D + c0 + j];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) g[e][j] += go;
+    }
+    bool clamped = false;
+    auto cexp = [&](float x) { if (x > 80.f) { clamped = true; x = 80.f; } return __expf(x); };
+    auto pack8 = [](const float *a) {
+        return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
+                          pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
+    };
+    auto unpack8 = [](const uint4 &u, float *a) {
+        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { a[2 * j] = __low2float(b[j]); a[2 * j + 1] = __high2float(b[j]); }
+    };
+    auto ld8 = [&](int row, float *a) {  // 8 per-channel constants of this octet
+        const float4 x = *reinterpret_cast<const float4 *>(cst + row * D + c0);
+        const float4 y = *reinterpret_cast<const float4 *>(cst + row * D + c0 + 4);
+        a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w; a[4] = y.x; a[5] = y.y; a[6] = y.z; a[7] = y.w;
+    };
+    const bool first_half = tg < 8;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int r = tg * 4 + e;
+        const uint32_t sw = ((ck ^ (uint32_t)(r & 7)) << 4);  // swizzled chunk offset
+        const float *ge = g[e];
+        const uint4 qe = qv[e], ke = kv[e], ve = vv[e];
+        float qf[8], kf[8], E[8], Hh[8], o[8];
+        unpack8(qe, qf); unpack8(ke, kf);
+        ld8(2, o);  // gC
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { E[j] = __expf(ge[j]); Hh[j] = __expf(o[j] - ge[j]); }
+        const float b = sbeta[r];
+        // record: Q~ (rows 64.. of A1) and K^ (MN-major image)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = qf[j] * E[j];
+        *reinterpret_cast<uint4 *>(rec + Record::kA1 + kb * 16384 + (64 + r) * 128 + sw) = pack8(o);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = kf[j] * Hh[j];
+        *reinterpret_cast<uint4 *>(rec + Record::kKh + kb * 8192 + r * 128 + sw) = pack8(o);
+        // solve right-hand sides (MN-major: token rows, channel columns)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = b * kf[j] * E[j];
+        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBK + kb * 8192 + r * 128 + sw) = pack8(o);
+        unpack8(ve, o);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] *= b;
+        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBV + kb * 8192 + r * 128 + sw) = pack8(o);
+        // factors for the A/P contraction: row factor -> E (in place), column
+        // factors -> Hh (in place) and o
+        float ref[8];
+        if (first_half) {
+            if (fast) {
+                ld8(3, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) E[j] *= ref[j];          // e^{g_r - g_15}
+                ld8(6, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = Hh[j] * ref[j];   // e^{g_31 - g_r}
+                ld8(5, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) Hh[j] *= ref[j];         // e^{g_15 - g_r}
+            } else {
+                ld8(0, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { E[j] = cexp(ge[j] - ref[j]); Hh[j] = cexp(ref[j] - ge[j]); }
+                ld8(1, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = cexp(ref[j] - ge[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { Hh[j] *= kf[j]; o[j] *= kf[j]; }
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + r * 128 + sw) = pack8(Hh);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + (32 + r) * 128 + sw) = pack8(o);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { o[j] = kf[j] * E[j]; qf[j] *= E[j]; }
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + r * 128 + sw) = pack8(o);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = pack8(qf);
+        } else {
+            if (fast) {
+                ld8(4, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) E[j] *= ref[j];          // e^{g_r - g_31}
+                ld8(6, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) Hh[j] *= ref[j];         // e^{g_31 - g_r}
+            } else {
+                ld8(1, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { E[j] = cexp(ge[j] - ref[j]); Hh[j] = cexp(ref[j] - ge[j]); }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { Hh[j] *= kf[j]; o[j] = kf[j] * E[j]; qf[j] *= E[j]; }
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + (32 + r) * 128 + sw) = pack8(Hh);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = pack8(o);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (64 + r) * 128 + sw) = pack8(qf);
+        }
+    }
+    // A chunk whose decay inside half a chunk exceeds the factorised range is
+    // recomputed exactly by the fixup kernel.
+    if (__syncthreads_or(clamped) && tid == 0) p.fix_list[atomicAdd(p.fix_count, 1)] = c * H + h;
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    tc::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- 2. MMA-AP
+    if (tid == 0) {
+        const uint32_t a0 = tc::smem_u32(sm + Prep2Smem::kAop);
+        const uint32_t b0 = tc::smem_u32(sm + Prep2Smem::kBop);
+        const uint32_t id = tc::idesc_bf16(128, 96, 0, 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = tc::smem_desc(a0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t b = tc::smem_desc(b0 + (kk >> 2) * 12288 + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(tmem, a, b, id, kk > 0);
+        }
+        tc::mma_commit(bar_ap);
+    }
+    float *As = reinterpret_cast<float *>(sm + Prep2Smem::kA);   // A[r][s], stride 65
+    float *Ts = reinterpret_cast<float *>(sm + Prep2Smem::kT);   // T[r][s], stride 65
+    float *Ys = reinterpret_cast<float *>(sm + Prep2Smem::kY);
+    {
+        // every warp reads its 32 TMEM lanes; warps 0-3 take the first 32 of the
+        // row's 64 relevant columns, warps 4-7 the other 32
+        tc::mbar_wait(bar_ap, 0, abort, p.err, 11);
+        tc::tc_fence_after_sync();
+        const int t = (warp & 3) * 32 + (tid & 31);  // accumulator row
+        const int sh = (warp >> 2) * 32;             // first s of this thread
+        const uint32_t col0 = (t < 64 ? 0u : 32u) + (uint32_t)sh;
+        float d[32];
+        tc::tmem_ld32_sync(tmem + ((uint32_t)((warp & 3) * 32) << 16) + col0, d);
+        const bool is_k = (t & 32) == 0;             // rows 0-31, 64-95 come from k
+        const int r = t < 64 ? (t & 31) : 32 + (t & 31);
+        const int lim = (t < 64) ? 32 : 64;          // first-half rows see only s < 32
+        if (is_k) {
+            const float b = sbeta[r];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int s2 = sh + e;
+                As[r * 65 + s2] = (s2 < lim && s2 < r) ? b * d[e] : 0.f;
+            }
+        } else {
+            uint8_t *prow = rec + Record::kP;
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int s0 = sh + c16 * 8 + 2 * e;
+                    w[e] = pack_bf16x2((s0 < lim && s0 <= r) ? d[c16 * 8 + 2 * e] : 0.f,
+                                       (s0 + 1 < lim && s0 + 1 <= r) ? d[c16 * 8 + 2 * e + 1] : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(prow + tc::sw128(r, (sh / 8 + c16) * 16)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+    tc::tc_fence_before_sync();
+    __syncthreads();
+
+    // ---- 3. T = (I + A)^{-1} by 16x16 blocks
+    {   // rows 64..127 of the [T; 0] operand are zero (this memory held the
+        // step-1 scratch until now)
+        uint4 *z = reinterpret_cast<uint4 *>(sm + Prep2Smem::kTt + 8192);
+        for (int i = tid; i < 8192 / 16; i += kPrep2Threads) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    if (tid < 64) {  // diagonal blocks: one column of one block per thread
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+            float acc = x[r];
+#pragma unroll
+            for (int s2 = 0; s2 < r; ++s2) acc -= As[(o + r) * 65 + o + s2] * x[s2];
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ts[(o + r) * 65 + o + cc] = x[r];
+    }
+    __syncthreads();
+    const int rr = tid >> 4, cc = tid & 15;
+    // distance 1: T_{i,i-1} = -T_ii (A_{i,i-1} T_{i-1,i-1}), i = 1..3
+    for (int i = 1; i < 4; ++i)
+        Ys[(i - 1) * 256 + rr * 16 + cc] =
+            blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), rr, cc);
+    __syncthreads();
+    for (int i = 1; i < 4; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            acc += Ts[(16 * i + rr) * 65 + 16 * i + k] * Ys[(i - 1) * 256 + k * 16 + cc];
+        Ts[(16 * i + rr) * 65 + 16 * (i - 1) + cc] = -acc;
+    }
+    __syncthreads();
+    // distance 2: T_{i,i-2} = -T_ii (A_{i,i-2} T_{i-2,i-2} + A_{i,i-1} T_{i-1,i-2}), i = 2, 3
+    for (int i = 2; i < 4; ++i)
+        Ys[(i - 2) * 256 + rr * 16 + cc] =
+            blk_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), rr, cc) +
+            blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), rr, cc);
+    __syncthreads();
+    for (int i = 2; i < 4; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            acc += Ts[(16 * i + rr) * 65 + 16 * i + k] * Ys[(i - 2) * 256 + k * 16 + cc];
+        Ts[(16 * i + rr) * 65 + 16 * (i - 2) + cc] = -acc;
+    }
+    __syncthreads();
+    // distance 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)
+    Ys[rr * 16 + cc] = blk_dot(As, 48, 0, Ts, 0, 0, rr, cc) +
+                       blk_dot(As, 48, 16, Ts, 16, 0, rr, cc) +
+                       blk_dot(As, 48, 32, Ts, 32, 0, rr, cc);
+    __syncthreads();
+    {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc += Ts[(48 + rr) * 65 + 48 + k] * Ys[k * 16 + cc];
+        Ts[(48 + rr) * 65 + cc] = -acc;
+    }
+    __syncthreads();
+    {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
+        const int r = tid >> 2, s0 = (tid & 3) * 16;
+        uint8_t *tt = sm + Prep2Smem::kTt;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int sa = s0 + h2 * 8 + 2 * e, sb2 = sa + 1;
+                const float va = sa < r ? Ts[r * 65 + sa] : (sa == r ? 1.f : 0.f);
+                const float vb = sb2 < r ? Ts[r * 65 + sb2] : (sb2 == r ? 1.f : 0.f);
+                w[e] = pack_bf16x2(va, vb);
+            }
+            *reinterpret_cast<uint4 *>(tt + tc::sw128(r, (s0 + h2 * 8) * 2)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    tc::tc_fence_after_sync();
+
+    // ---- 4. [W | U~] = [T; 0] . [beta K~ | beta V]
+    if (tid == 0) {
+        const uint32_t bkv = tc::smem_u32(sm + Prep2Smem::kBK);  // 4 MN atoms: BK then BV
+        const uint32_t tt = tc::smem_u32(sm + Prep2Smem::kTt);
+        const uint32_t id = tc::idesc_bf16(128, 256, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem, tc::smem_desc(tt + kk * 32, 16, 1024),
+                         tc::smem_desc(bkv + kk * 2048, 8192, 1024), id, kk > 0);
+        tc::mma_commit(bar_wu);
+    }
+    if ((warp & 3) < 2) {  // warps 0,1: W (columns 0..127); warps 4,5: U~ (128..255)
+        tc::mbar_wait(bar_wu, 0, abort, p.err, 12);
+        tc::tc_fence_after_sync();
+        const int r = (warp & 3) * 32 + (tid & 31);  // token
+        const uint32_t la = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        float w[32];
+        if (warp < 4) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                tc::tmem_ld32_sync(la + q4 * 32, w);
+                uint8_t *a1 = rec + Record::kA1 + (uint32_t)(q4 >> 1) * 16384;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
+                    *reinterpret_cast<uint4 *>(a1 + tc::sw128(r, ((q4 & 1) * 4 + c16) * 16)) =
+                        make_uint4(u[0], u[1], u[2], u[3]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                tc::tmem_ld32_sync(la + 128 + q4 * 32, w);
+                uint8_t *uu = rec + Record::kU + (uint32_t)(q4 >> 1) * 16384;
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    *reinterpret_cast<float4 *>(uu + u_swz(r, (q4 & 1) * 32 + 4 * m)) =
+                        make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+            }
+        }
+    }
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
     }
 }
 
@@ -403,6 +868,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
 }
 
 constexpr size_t kPrepSmem = sizeof(float) * (3 * C * (D + 1) + C * D + C * (C + 1) + C);
+constexpr int kFixupBlocks = 148;
 
 }  // namespace
 
@@ -414,8 +880,9 @@ bool tc_supported(const Problem &p)
 WorkspaceLayout tc_workspace_layout(const Problem &p)
 {
     WorkspaceLayout l;
-    // plan arrays + the device error word
-    l.plan_bytes = align_up(sizeof(int32_t) * (2 * (size_t)(p.N + 1) + 1), 1024);
+    // plan arrays, the error word, the fixup count and the fixup list
+    l.plan_bytes = align_up(sizeof(int32_t) * (2 * (size_t)(p.N + 1) + 2 +
+                                               (size_t)p.max_chunks * p.H), 1024);
     l.chunk_bytes = (size_t)Record::kBytes * (size_t)p.H * (size_t)p.max_chunks;
     l.total = l.plan_bytes + l.chunk_bytes;
     return l;
@@ -436,19 +903,27 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
     plan.chunk_off = plan.seq_start + (pb.N + 1);
     p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off;
     p.err = plan.chunk_off + (pb.N + 1);
+    p.fix_count = p.err + 1;
+    p.fix_list = p.err + 2;
     p.rec = static_cast<uint8_t *>(workspace) + lay.plan_bytes;
 
     cudaError_t e = cudaSuccess;
     if (phases & kPhasePrepare) {
         e = launch_plan(pb, plan, st);
         if (e != cudaSuccess) return e;
-        e = cudaMemsetAsync(p.err, 0, sizeof(int), st);
+        e = cudaMemsetAsync(p.err, 0, 2 * sizeof(int), st);
         if (e != cudaSuccess) return e;
         if (pb.max_chunks > 0) {
-            e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kPrepSmem);
+            e = cudaFuncSetAttribute(tc_prep2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)Prep2Smem::kBytes);
             if (e != cudaSuccess) return e;
-            tc_prep_kernel<<<dim3(pb.max_chunks, pb.H), kPrepThreads, kPrepSmem, st>>>(p);
+            tc_prep2_kernel<<<dim3(pb.max_chunks, pb.H), kPrep2Threads, Prep2Smem::kBytes, st>>>(p);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(tc_prep_fixup_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
+            if (e != cudaSuccess) return e;
+            tc_prep_fixup_kernel<<<kFixupBlocks, kPrepThreads, kPrepSmem, st>>>(p);
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }

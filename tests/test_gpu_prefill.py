@@ -174,3 +174,31 @@ def test_prepare_then_carry_equals_one_call(algo):
     call = kda.kda_chunk_fwd_prepare(*a, algo=algo)
     o2, S2 = kda.kda_chunk_fwd_carry(call)
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+@pytest.mark.parametrize("algo", ["simt", "tcgen05"])
+@pytest.mark.parametrize("gate_shift", [1.0, 3.0])
+def test_strong_decay_gates(algo, gate_shift):
+    """Fast-forgetting gates: log_alpha = -softplus(N(0,1) + shift). With shift 1 a
+    chunk decays by ~80 nats (the tensor-core prep switches to direct
+    exponentials); with shift 3 half a chunk decays by ~100 nats (the chunk is
+    recomputed by the exact fixup). Results must match the oracle either way."""
+    _skip_unless(algo)
+    x = I.make_prefill(2, 300, 3, 128, torch.bfloat16, gate_shift=gate_shift, s0_std=0.05,
+                       seed=41)
+    o, Sf, o_ref, S_ref = run_both(x, algo=algo)
+    assert rel_l2(o, o_ref) <= 2e-2
+    assert rel_l2(Sf, S_ref) <= 2e-2
+
+
+@pytest.mark.parametrize("gate_shift", [-3.0, 0.0, 3.0])
+def test_tcgen05_matches_simt(gate_shift):
+    """The two GPU paths agree with each other on the same inputs."""
+    if not _has_tc():
+        pytest.skip("tcgen05 path not built")
+    x = to_cuda(I.make_prefill(2, 333, 4, 128, torch.bfloat16, gate_shift, 0.05, seed=42))
+    a = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
+    o1, S1 = kda.kda_chunk_fwd(*a, algo="simt")
+    o2, S2 = kda.kda_chunk_fwd(*a, algo="tcgen05")
+    assert rel_l2(o2, o1.double().cpu().numpy()) <= 2e-2
+    assert rel_l2(S2, S1.double().cpu().numpy()) <= 2e-2
