@@ -1,0 +1,61 @@
+// kda_noalloc.cu — kda_chunk_fwd for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc: a plugin whose host application owns all
+// device memory and hands out none, or code running where an allocation's
+// implicit device synchronisation is not allowed. kda_chunk_fwd_noalloc serves
+// them: it runs the same prefill as kda_chunk_fwd_ex, but its workspace is a
+// fixed array in the library's own device memory instead of a caller buffer.
+//
+// The array is a file-scope __device__ variable of KDA_NOALLOC_SCRATCH_BYTES.
+// Every GPU that loads the library holds it until the process exits. Host code
+// cannot pass the variable's name to a kernel (on the host the name is only a
+// stand-in, not a device address), so the first call on each device looks up
+// the device address with cudaGetSymbolAddress, with that device current, and
+// caches it; later calls on that device reuse it.
+#include <mutex>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+
+// Device address of the scratch array on the current device (set up once).
+cudaError_t scratch_on_current_device(void **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" kda_status_t kda_chunk_fwd_noalloc(
+    const void *q, const void *k, const void *v, kda_dtype_t dt, const float *log_alpha,
+    const float *beta, const float *S0, const int32_t *cu_seqlens, int n_seqs, int B, int T,
+    int H, int dk, int dv, float scale, void *o, float *S_final, int algo, void *stream)
+{
+    // The size limit is checked on the host before any CUDA call.
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv,
+                                                     cu_seqlens ? n_seqs : 0, dt);
+    if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (scratch_on_current_device(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+    return kda_chunk_fwd_ex(q, k, v, dt, log_alpha, beta, S0, cu_seqlens, n_seqs, B, T, H,
+                            dk, dv, scale, o, S_final, scratch, KDA_NOALLOC_SCRATCH_BYTES, algo,
+                            stream);
+}

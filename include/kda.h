@@ -161,6 +161,38 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dt
                              const float *log_alpha, const float *beta, float *S, int N,
                              int H, int dk, int dv, float scale, void *o, void *stream);
 
+/*
+ * kda_chunk_fwd_noalloc — the chunked prefill for callers that cannot allocate
+ * device memory (no counterpart in the paper; it exists for callers such as a
+ * plugin whose host application owns all device memory, or code that must not
+ * trigger the device synchronisation an allocation can cause).
+ *
+ * Same arguments and results as kda_chunk_fwd_ex, minus the workspace: the
+ * library uses a fixed scratch array of KDA_NOALLOC_SCRATCH_BYTES in its own
+ * device memory, held by every GPU that loads the library until the process
+ * exits. The caller still provides every input and output buffer. The call
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
+ *   - Problems whose workspace (kda_chunk_fwd_workspace_size) exceeds
+ *     KDA_NOALLOC_SCRATCH_BYTES are rejected on the host with
+ *     KDA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress, with that device current); make that
+ *     first call before any stream capture on the device.
+ *   - Every call shares the one array and leaves its contents behind. The
+ *     kernels initialise every part of it they read, so nothing carries over
+ *     from one call to the next; but calls whose execution overlaps on the GPU
+ *     (different streams, or different host threads) race on the array and
+ *     must be serialised by the caller.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                   kda_dtype_t qkv_dtype, const float *log_alpha,
+                                   const float *beta, const float *S0,
+                                   const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                                   int dk, int dv, float scale, void *o, float *S_final,
+                                   int algo, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
