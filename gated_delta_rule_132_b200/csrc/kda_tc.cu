@@ -659,10 +659,23 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
 }
 
 // ------------------------------------------------------------------- carry
-constexpr int kCarryThreads = 192;  // warps 0-3 epilogue, 4 producer, 5 MMA
-constexpr uint32_t kTmemCols = 128; // D1: columns [0,64), D2: [64,128)
+// Warps 0-7 (256 threads) own the 128 x 64 state slice: warp w serves TMEM lanes
+// 32*(w%4).. (state rows) and value columns 32*(w/4).. of the slice, so each
+// thread keeps one state row x 32 columns in fp32 registers. Warp 8 streams
+// records. Thread 0 issues each MMA group right after the named barrier that
+// completes its operands, so the waits on the critical path are the two MMA
+// completions per chunk plus the epilogues. The output accumulator D1 is
+// double-buffered in TMEM, so the output rows of chunk c are read (warps
+// serving lanes 64..127) after chunk c+1's first MMA group is already issued.
+constexpr int kCarryThreads = 288;
+constexpr uint32_t kTmemCols = 256;  // D1[0]: [0,64), D2: [64,128), D1[1]: [128,192)
 
-enum { kErrFull = 1, kErrEmpty, kErrD1, kErrU, kErrD2, kErrS };
+enum { kErrFull = 1, kErrEmpty, kErrD1, kErrD2 };
+
+__device__ __forceinline__ void named_bar(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
 {
@@ -673,29 +686,26 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     uint64_t *full = bars + 0;   // [2]
     uint64_t *empty = bars + 2;  // [2]
     uint64_t *d1_done = bars + 4;
-    uint64_t *u_ready = bars + 5;
-    uint64_t *d2_done = bars + 6;
-    uint64_t *s_ready = bars + 7;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 9);
+    uint64_t *d2_done = bars + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 7);
 
     const int n = blockIdx.x, h = blockIdx.y, half = blockIdx.z, H = p.H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&full[0], 1); tc::mbar_init(&full[1], 1);
-        tc::mbar_init(&empty[0], 4); tc::mbar_init(&empty[1], 4);
-        tc::mbar_init(d1_done, 1); tc::mbar_init(u_ready, 2);
-        tc::mbar_init(d2_done, 1); tc::mbar_init(s_ready, 4);
+        tc::mbar_init(&empty[0], 8); tc::mbar_init(&empty[1], 8);
+        tc::mbar_init(d1_done, 1); tc::mbar_init(d2_done, 1);
         *abort = 0;
         tc::fence_mbar_init();
     }
     // rows 0..63 of the [0; P] operand stay zero
-    for (int s = 0; s < 2; ++s) {
-        uint4 *z = reinterpret_cast<uint4 *>(sm + s * CarrySmem::kStage + CarrySmem::kA2b);
+    for (int s2 = 0; s2 < 2; ++s2) {
+        uint4 *z = reinterpret_cast<uint4 *>(sm + s2 * CarrySmem::kStage + CarrySmem::kA2b);
         for (int i = threadIdx.x; i < 8192 / 16; i += kCarryThreads) z[i] = make_uint4(0, 0, 0, 0);
     }
-    if (warp == 5) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
+    if (warp == 0) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
@@ -705,7 +715,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     const int ts = p.seq_start[n], te = p.seq_start[n + 1];
     const int c0 = p.chunk_off[n], nc = p.chunk_off[n + 1] - c0;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------- producer: one record per chunk into the two-stage ring
         if (lane == 0) {
             for (int lc = 0; lc < nc; ++lc) {
@@ -724,144 +734,144 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             for (int lc = (nc > 2 ? nc - 2 : 0); lc < nc; ++lc)
                 tc::mbar_wait(&full[lc & 1], (lc >> 1) & 1, abort, p.err, kErrFull);
         }
-    } else if (warp == 5) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 1);   // [W;Q~] K-major . S MN-major
-            const uint32_t id2a = tc::idesc_bf16(128, 64, 1, 1);  // K^^T MN-major . U MN-major
-            const uint32_t id2b = tc::idesc_bf16(128, 64, 0, 1);  // [0;P] K-major . U MN-major
-            const uint32_t b1 = tc::smem_u32(sm + CarrySmem::kB1);
-            const uint32_t b2 = tc::smem_u32(sm + CarrySmem::kB2);
-            for (int lc = 0; lc < nc; ++lc) {
-                const int st = lc & 1;
-                const uint32_t sb = tc::smem_u32(sm + st * CarrySmem::kStage);
-                tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
-                tc::mbar_wait(s_ready, lc & 1, abort, p.err, kErrS);
-                tc::tc_fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = tc::smem_desc(sb + CarrySmem::kA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = tc::smem_desc(b1 + kk * 2048, 8192, 1024);
-                    tc::mma_bf16(tmem + 0, a, b, id1, kk > 0);
-                }
-                tc::mma_commit(d1_done);
-                tc::mbar_wait(u_ready, lc & 1, abort, p.err, kErrU);
-                tc::tc_fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = tc::smem_desc(sb + CarrySmem::kKh + kk * 2048, 8192, 1024);
-                    const uint64_t b = tc::smem_desc(b2 + kk * 2048, 8192, 1024);
-                    tc::mma_bf16(tmem + 64, a, b, id2a, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = tc::smem_desc(sb + CarrySmem::kA2b + kk * 32, 16, 1024);
-                    const uint64_t b = tc::smem_desc(b2 + kk * 2048, 8192, 1024);
-                    tc::mma_bf16(tmem + 0, a, b, id2b, 1);
-                }
-                tc::mma_commit(d2_done);
-            }
-        }
     } else {
-        // ---------------- epilogue: thread t owns row t of the state slice
-        const int t = threadIdx.x;  // 0..127
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        float S[kSlice];
-        const size_t sbase = (((size_t)n * H + h) * D + t) * D + half * kSlice;
+        // ---------------- state owners
+        const int lg = warp & 3;                  // TMEM lane group
+        const int t = lg * 32 + lane;             // state row (dk index) / accumulator row
+        const int cb = (warp >> 2) * 32;          // first value column of this thread
+        const uint32_t lane_addr = tmem + ((uint32_t)(lg * 32) << 16);
+        const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 1);   // [W;Q~] K-major . S MN-major
+        const uint32_t id2a = tc::idesc_bf16(128, 64, 1, 1);  // K^^T MN-major . U MN-major
+        const uint32_t id2b = tc::idesc_bf16(128, 64, 0, 1);  // [0;P] K-major . U MN-major
+        const uint32_t b1 = tc::smem_u32(sm + CarrySmem::kB1);
+        const uint32_t b2 = tc::smem_u32(sm + CarrySmem::kB2);
+        float S[32];
+        const size_t sbase = (((size_t)n * H + h) * D + t) * D + half * kSlice + cb;
 #pragma unroll
-        for (int j = 0; j < kSlice; j += 4) {
+        for (int j = 0; j < 32; j += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (p.S0) x = *reinterpret_cast<const float4 *>(p.S0 + sbase + j);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        uint8_t *b1row = sm + CarrySmem::kB1;
-        auto store_row_bf16 = [&](uint8_t *base, int row, const float *vals) {
+        // bf16 copy of this thread's 32 values into row `row` of a 64-column
+        // MN-major operand (4 of the row's 8 swizzled 16-byte chunks)
+        auto store_bf16 = [&](uint8_t *base, int row, const float *vals) {
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                __nv_bfloat162 w[4];
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t w[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w[e] = __floats2bfloat162_rn(vals[c16 * 8 + 2 * e], vals[c16 * 8 + 2 * e + 1]);
-                *reinterpret_cast<uint4 *>(base + tc::sw128(row, c16 * 16)) =
-                    *reinterpret_cast<uint4 *>(w);
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 b = __floats2bfloat162_rn(vals[c4 * 8 + 2 * e],
+                                                             vals[c4 * 8 + 2 * e + 1]);
+                    w[e] = *reinterpret_cast<uint32_t *>(&b);
+                }
+                *reinterpret_cast<uint4 *>(base + tc::sw128(row, (cb / 8 + c4) * 16)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
-        store_row_bf16(b1row, t, S);
+        // output rows of chunk lc (lanes 64..127): D1[lc & 1] -> o
+        auto write_o = [&](int lc) {
+            const int r = t - 64;
+            const int t0 = ts + lc * C;
+            float ov[32];
+            tc::tmem_ld32_sync(lane_addr + (lc & 1) * 128 + cb, ov);
+            if (r < min(C, te - t0)) {
+                __nv_bfloat16 *orow = p.o + ((size_t)(t0 + r) * H + h) * D + half * kSlice + cb;
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(p.scale * ov[j + 2 * e],
+                                                                 p.scale * ov[j + 2 * e + 1]);
+                        w[e] = *reinterpret_cast<uint32_t *>(&b);
+                    }
+                    *reinterpret_cast<uint4 *>(orow + j) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        };
+        store_bf16(sm + CarrySmem::kB1, t, S);
         tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(s_ready);
+        tc::tc_fence_before_sync();
 
         for (int lc = 0; lc < nc; ++lc) {
             const int st = lc & 1;
             uint8_t *sb = sm + st * CarrySmem::kStage;
-            const int t0 = ts + lc * C;
-            const int L = min(C, te - t0);
+            const uint32_t d1 = tmem + (uint32_t)st * 128;  // this chunk's output accumulator
+            // A. the bf16 state is complete: issue MMA1 = [W; Q~] . S
+            named_bar(1, 256);
+            if (threadIdx.x == 0) {
+                tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
+                tc::tc_fence_after_sync();
+                const uint32_t sbase_a = tc::smem_u32(sb + CarrySmem::kA1);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(d1, tc::smem_desc(sbase_a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                 tc::smem_desc(b1 + kk * 2048, 8192, 1024), id1, kk > 0);
+                tc::mma_commit(d1_done);
+            }
+            // E. previous chunk's output rows, off the critical path
+            if (lg >= 2 && lc > 0) write_o(lc - 1);
             tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
-            if (warp < 2) {
+            if (lg < 2) {
+                // C. U = U~ - W S for tokens 0..63, then MMA2
                 tc::mbar_wait(d1_done, lc & 1, abort, p.err, kErrD1);
                 tc::tc_fence_after_sync();
-                float U[kSlice];
-                tc::tmem_ld32_sync(lane_addr + 0, U);
-                tc::tmem_ld32_sync(lane_addr + 32, U + 32);
+                float U[32];
+                tc::tmem_ld32_sync(lane_addr + (uint32_t)st * 128 + cb, U);
 #pragma unroll
-                for (int j = 0; j < kSlice; j += 4) {
+                for (int j = 0; j < 32; j += 4) {
                     const float4 ut = *reinterpret_cast<const float4 *>(
-                        sb + CarrySmem::kU + u_swz(t, j));
-                    U[j] = ut.x - U[j];
-                    U[j + 1] = ut.y - U[j + 1];
-                    U[j + 2] = ut.z - U[j + 2];
-                    U[j + 3] = ut.w - U[j + 3];
+                        sb + CarrySmem::kU + u_swz(t, cb + j));
+                    U[j] = ut.x - U[j]; U[j + 1] = ut.y - U[j + 1];
+                    U[j + 2] = ut.z - U[j + 2]; U[j + 3] = ut.w - U[j + 3];
                 }
-                store_row_bf16(sm + CarrySmem::kB2, t, U);
+                store_bf16(sm + CarrySmem::kB2, t, U);
                 tc::fence_proxy_async_smem();
                 tc::tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(u_ready);
-            }
-            tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2);
-            tc::tc_fence_after_sync();
-            const float gamma = reinterpret_cast<const float *>(sb + CarrySmem::kG)[t];
-            {
-                float ku[kSlice];
-                tc::tmem_ld32_sync(lane_addr + 64, ku);
-                tc::tmem_ld32_sync(lane_addr + 96, ku + 32);
+                named_bar(2, 128);
+                if (threadIdx.x == 0) {
+                    tc::tc_fence_after_sync();
+                    const uint32_t kh = tc::smem_u32(sb + CarrySmem::kKh);
+                    const uint32_t a2b = tc::smem_u32(sb + CarrySmem::kA2b);
 #pragma unroll
-                for (int j = 0; j < kSlice; ++j) S[j] = gamma * S[j] + ku[j];
-            }
-            store_row_bf16(b1row, t, S);
-            if (warp >= 2) {
-                const int r = t - 64;
-                __nv_bfloat16 *orow = p.o + ((size_t)(t0 + r) * H + h) * D + half * kSlice;
-                float ov[kSlice];
-                tc::tmem_ld32_sync(lane_addr + 0, ov);
-                tc::tmem_ld32_sync(lane_addr + 32, ov + 32);
-                if (r < L) {
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tmem + 64, tc::smem_desc(kh + kk * 2048, 8192, 1024),
+                                     tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2a, kk > 0);
 #pragma unroll
-                    for (int j = 0; j < kSlice; j += 8) {
-                        __nv_bfloat162 w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = __floats2bfloat162_rn(p.scale * ov[j + 2 * e],
-                                                         p.scale * ov[j + 2 * e + 1]);
-                        *reinterpret_cast<uint4 *>(orow + j) = *reinterpret_cast<uint4 *>(w);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(d1, tc::smem_desc(a2b + kk * 32, 16, 1024),
+                                     tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2b, 1);
+                    tc::mma_commit(d2_done);
                 }
             }
+            // D. S = gamma * S + K^^T U, and its bf16 copy for the next MMA1
+            tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2);
+            tc::tc_fence_after_sync();
+            {
+                float ku[32];
+                tc::tmem_ld32_sync(tmem + 64 + ((uint32_t)(lg * 32) << 16) + cb, ku);
+                const float gamma = reinterpret_cast<const float *>(sb + CarrySmem::kG)[t];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = gamma * S[j] + ku[j];
+            }
+            store_bf16(sm + CarrySmem::kB1, t, S);
             tc::fence_proxy_async_smem();
             tc::tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) { tc::mbar_arrive(s_ready); tc::mbar_arrive(&empty[st]); }
+            if (lane == 0) tc::mbar_arrive(&empty[st]);
         }
+        if (lg >= 2 && nc > 0) write_o(nc - 1);
         if (p.S_final) {
 #pragma unroll
-            for (int j = 0; j < kSlice; j += 4)
+            for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4 *>(p.S_final + sbase + j) =
                     make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     }
     tc::tc_fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 0) {
         tc::tc_fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
