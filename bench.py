@@ -39,6 +39,12 @@ METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM pea
 # Kernels one tcgen05 prefill call launches: plan, prep, exact fixup (exits at
 # once when no chunk needs it), carry. (The error-word reset is a memset.)
 LAUNCHES_PER_PREFILL = 4
+# DRAM traffic per (chunk, head) record measured by ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum) on the chunked workload, one launch of 4096 records;
+# traffic grows in proportion to the records a launch processes. Sources:
+# profiles/tc_prep2_kernel_chunked_B4_H16_T4096.md and
+# profiles/tc_carry_kernel_chunked_B4_H16_T4096.md.
+TRAFFIC_PER_RECORD = {"prepare": 162_723, "carry": 106_143}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -193,9 +199,15 @@ def bench_prefill(preset, steps, warmup, world, rank, dev, peaks):
     state_b = n_seq * preset.H * d * d * 4 * (2 if x["S0"] is not None else 1)
     op_bytes = token_heads * (in_b + out_b) + state_b
     ws_bytes = call.workspace.numel()
+    if x["cu_seqlens"] is None:
+        chunks = preset.B * ((x["q"].shape[1] + 63) // 64)
+    else:
+        cu = x["cu_seqlens"].cpu().tolist()
+        chunks = sum((cu[i + 1] - cu[i] + 63) // 64 for i in range(len(cu) - 1))
     return dict(x=x, call=call, ms=ms, prep_ms=prep_ms, carry_ms=carry_ms, tokens=tokens,
                 token_heads=token_heads, op_bytes=op_bytes, in_bytes=token_heads * in_b,
-                out_bytes=token_heads * out_b + state_b, ws_bytes=ws_bytes)
+                out_bytes=token_heads * out_b + state_b, ws_bytes=ws_bytes,
+                records=chunks * preset.H)
 
 
 def bench_decode(P, steps, warmup, world, rank, dev):
@@ -294,7 +306,9 @@ def run_ours(args, world, rank, dev):
     hbm = peaks["hbm_gbs"]
     value = pre["tokens"] * world / (pre["ms"] / 1e3)
 
-    # Dominant prefill kernel and its roofline (HBM: bytes it must move / its time).
+    # Dominant prefill kernel and its roofline (HBM: the bytes it must move, i.e.
+    # its inputs plus the per-chunk records it writes (prepare) or reads
+    # (carry) plus its outputs, over its measured time).
     ws_per_launch = pre["ws_bytes"]
     prep_bytes = pre["in_bytes"] + ws_per_launch
     carry_bytes = ws_per_launch + pre["out_bytes"]
@@ -305,7 +319,9 @@ def run_ours(args, world, rank, dev):
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     ach = kernels[dom]["bytes"] / (kernels[dom]["ms"] / 1e3) / 1e9
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-            "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": None,
+            "unit": "GB/s", "frac": round(ach / hbm, 4),
+            "traffic": TRAFFIC_PER_RECORD[dom] * pre["records"],
+            "traffic_note": "ncu DRAM bytes per record on the chunked workload x records",
             "peak_source": peak_kind,
             "bytes_per_launch": kernels[dom]["bytes"], "ms_per_launch": kernels[dom]["ms"]}
     op_ach = pre["op_bytes"] / (pre["ms"] / 1e3) / 1e9
@@ -326,6 +342,8 @@ def run_ours(args, world, rank, dev):
                         "note": "algorithmic bytes of the whole prefill (q,k,v,log_alpha,"
                                 "beta in, o out, states) / step time"},
         "kernels_ms": {n: round(v["ms"], 4) for n, v in kernels.items()},
+        "kernels_roofline_frac": {n: round(v["bytes"] / (v["ms"] / 1e3) / 1e9 / hbm, 4)
+                                  for n, v in kernels.items()},
         "gpu_launches": LAUNCHES_PER_PREFILL * args.steps,
     }
     if dec is not None:
@@ -382,7 +400,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": preset.name, "B": preset.B, "T": int(pre["tokens"]), "H": preset.H,
+        "config": {"workload": preset.name, "B": preset.B, "T": preset.T, "H": preset.H,
                    "d_k": preset.d, "d_v": preset.d},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": used,
                          "kind": "oracle", "sample": sample},

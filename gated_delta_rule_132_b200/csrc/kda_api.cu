@@ -63,19 +63,22 @@ const char *kda_status_string(kda_status_t s)
 
 int kda_version(void) { return 100; }
 
-size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
-                                    kda_dtype_t dt)
+size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
+                                       kda_dtype_t dt, int algo)
 {
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TCGEN05) return 0;
     kda::Problem p;
     const bool varlen = n_seqs > 0 && B == 1;
     if (describe(B, T, H, dk, dv, n_seqs, varlen, dt, &p) != KDA_OK) return 0;
-    // Enough for whichever path kda_chunk_fwd selects (and for the SIMT path).
-    size_t s = required_bytes(p, false);
-    if (kda::tc_supported(p)) {
-        const size_t t = required_bytes(p, true);
-        if (t > s) s = t;
-    }
-    return s;
+    const bool tc = use_tc(p, algo);
+    if (algo == KDA_ALGO_TCGEN05 && !tc) return 0;
+    return required_bytes(p, tc);
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                    kda_dtype_t dt)
+{
+    return kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, n_seqs, dt, KDA_ALGO_AUTO);
 }
 
 }  // extern "C"

@@ -50,8 +50,8 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(
     int H, int dk, int dv, float scale, void *o, float *S_final, int algo, void *stream)
 {
     // The size limit is checked on the host before any CUDA call.
-    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv,
-                                                     cu_seqlens ? n_seqs : 0, dt);
+    const size_t need = kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv,
+                                                        cu_seqlens ? n_seqs : 0, dt, algo);
     if (need > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
     void *scratch = nullptr;
     if (scratch_on_current_device(&scratch) != cudaSuccess) return KDA_ERR_CUDA;

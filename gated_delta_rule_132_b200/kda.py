@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.kda_version.argtypes = []
         L.kda_chunk_fwd_workspace_size.restype = _sz
         L.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
+        L.kda_chunk_fwd_workspace_size_ex.restype = _sz
+        L.kda_chunk_fwd_workspace_size_ex.argtypes = [_i] * 8
         common = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                   _vp, _vp, _vp, _sz]
         L.kda_chunk_fwd.restype = _i
@@ -95,10 +97,12 @@ def _need(t, name, dtype=None, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs=0, dtype=torch.bfloat16) -> int:
-    """Bytes of workspace :func:`kda_chunk_fwd` needs (C: same name)."""
+def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs=0, dtype=torch.bfloat16,
+                                 algo="auto") -> int:
+    """Bytes of workspace :func:`kda_chunk_fwd` needs with ``algo``
+    (C: ``kda_chunk_fwd_workspace_size_ex``)."""
     d = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
-    return int(lib().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs, d))
+    return int(lib().kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, n_seqs, d, ALGOS[algo]))
 
 
 class ChunkFwdCall:
@@ -137,7 +141,7 @@ class ChunkFwdCall:
         elif S_final is not None:
             _need(S_final, "S_final", torch.float32, (N, H, dk, dv))
         n_seqs = N if cu_seqlens is not None else 0
-        need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs, dtype)
+        need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, n_seqs, dtype, algo)
         if workspace is None:
             workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
         self.tensors = (q, k, v, log_alpha, beta, S0, cu_seqlens, workspace)

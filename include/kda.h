@@ -75,8 +75,8 @@ const char *kda_status_string(kda_status_t status);
 int kda_version(void);
 
 /*
- * Workspace bytes that kda_chunk_fwd needs for this problem (0 on invalid
- * sizes). The workspace holds the per-chunk intermediate matrices of the
+ * Workspace bytes that kda_chunk_fwd needs for this problem, i.e. for the path
+ * KDA_ALGO_AUTO selects (0 on invalid sizes). The workspace holds the per-chunk intermediate matrices of the
  * chunked form between the chunk-parallel and the sequential kernel; it is
  * device memory owned by the caller, needs no initialisation and may be reused
  * across calls on the same stream. For varlen calls pass B = 1, T = total
@@ -84,6 +84,12 @@ int kda_version(void);
  */
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
                                     kda_dtype_t qkv_dtype);
+
+/* Workspace bytes kda_chunk_fwd_ex needs with the given kda_algo_t (the size for
+ * the path that algo selects; KDA_ALGO_AUTO gives the same value as
+ * kda_chunk_fwd_workspace_size). 0 on invalid sizes or an unsupported algo. */
+size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
+                                       kda_dtype_t qkv_dtype, int algo);
 
 /*
  * Chunked prefill: runs the recurrence over every sequence from S0 (NULL = zero

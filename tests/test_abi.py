@@ -102,3 +102,16 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         kda.lib()
+
+
+def test_workspace_size_per_algorithm(L):
+    """The tcgen05 path needs less workspace than the SIMT path; asking for a
+    path a problem does not support gives 0."""
+    L.kda_chunk_fwd_workspace_size_ex.restype = ctypes.c_size_t
+    tc = L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 128, 128, 0, 1, 2)
+    simt = L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 128, 128, 0, 1, 1)
+    auto = L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 128, 128, 0, 1, 0)
+    assert 0 < tc < simt and auto == tc
+    assert L.kda_chunk_fwd_workspace_size(1, 4096, 8, 128, 128, 0, 1) == tc
+    assert L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 64, 64, 0, 1, 2) == 0
+    assert L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 128, 128, 0, 1, 7) == 0
