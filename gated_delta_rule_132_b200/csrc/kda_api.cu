@@ -24,6 +24,7 @@ kda_status_t describe(int B, int T, int H, int dk, int dv, int n_seqs, bool varl
     const long long total = (long long)B * T;
     if (total > (long long)INT32_MAX - kda::kChunk) return KDA_ERR_UNSUPPORTED;
     const int N = varlen ? n_seqs : B;
+    if ((long long)N * H * 4 > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;  // carry grid
     long long chunks = varlen ? total / kda::kChunk + N
                               : (long long)B * ((T + kda::kChunk - 1) / kda::kChunk);
     if (chunks > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;

@@ -41,11 +41,17 @@ struct Problem {
 
 // Sequence plan in the workspace: for n in [0, N], the sanitised packed start
 // token seq_start[n] and first global chunk chunk_off[n] (both int32; entry N
-// holds the totals).
+// holds the totals), and order[0..N): the sequences by decreasing length, the
+// order in which the sequential kernels take them (longest first keeps the
+// last wave of CTAs short).
 struct Plan {
     int32_t *seq_start;
     int32_t *chunk_off;
+    int32_t *order;
 };
+
+// int32 entries of a plan for N sequences.
+inline size_t plan_ints(int N) { return 3 * (size_t)N + 2; }
 
 // Byte layout of one prefill workspace.
 struct WorkspaceLayout {

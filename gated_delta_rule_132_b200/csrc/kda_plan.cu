@@ -11,12 +11,18 @@
 // For well-formed input this changes nothing; for malformed input it keeps
 // every later access inside the caller's buffers and the chunk count within
 // floor(total / 64) + N, the bound the workspace is sized for.
+//
+// It also ranks the sequences by decreasing length (ties by index): the
+// sequential kernels take them in that order, so the longest sequences start
+// in the first wave of CTAs. Ranking is quadratic, so it is done for up to
+// kRankMax sequences; beyond that the order is the identity.
 #include "kda_internal.cuh"
 
 namespace kda {
 namespace {
 
 constexpr int kPlanThreads = 1024;
+constexpr int kRankMax = 2048;
 
 template <typename Op>
 __device__ int block_inclusive_scan(int x, Op op, int identity, int *s_warp)
@@ -49,15 +55,18 @@ struct AddOp { __device__ int operator()(int a, int b) const { return a + b; } }
 
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int32_t *__restrict__ cu_seqlens, int N, int T, int total,
-            int32_t *__restrict__ seq_start, int32_t *__restrict__ chunk_off)
+            int32_t *__restrict__ seq_start, int32_t *__restrict__ chunk_off,
+            int32_t *__restrict__ order)
 {
     __shared__ int s_warp[32];
     __shared__ int s_carry;
+    __shared__ int s_len[kRankMax];
     if (cu_seqlens == nullptr) {
         const int per = (T + kChunk - 1) / kChunk;
         for (int n = threadIdx.x; n <= N; n += kPlanThreads) {
             seq_start[n] = n * T;
             chunk_off[n] = n * per;
+            if (n < N) order[n] = n;
         }
         return;
     }
@@ -88,6 +97,22 @@ plan_kernel(const int32_t *__restrict__ cu_seqlens, int N, int T, int total,
         if (threadIdx.x == kPlanThreads - 1) s_carry = carry + incl;
         __syncthreads();
     }
+    // Pass 3: longest-first order.
+    if (N > kRankMax) {
+        for (int n = threadIdx.x; n < N; n += kPlanThreads) order[n] = n;
+        return;
+    }
+    for (int n = threadIdx.x; n < N; n += kPlanThreads) s_len[n] = seq_start[n + 1] - seq_start[n];
+    __syncthreads();
+    for (int n = threadIdx.x; n < N; n += kPlanThreads) {
+        const int ln = s_len[n];
+        int rank = 0;
+        for (int m = 0; m < N; ++m) {
+            const int lm = s_len[m];
+            rank += (lm > ln) || (lm == ln && m < n);
+        }
+        order[rank] = n;
+    }
 }
 
 }  // namespace
@@ -95,7 +120,7 @@ plan_kernel(const int32_t *__restrict__ cu_seqlens, int N, int T, int total,
 cudaError_t launch_plan(const Problem &p, Plan plan, cudaStream_t stream)
 {
     plan_kernel<<<1, kPlanThreads, 0, stream>>>(p.cu_seqlens, p.N, p.T, (int)p.total_tokens,
-                                                plan.seq_start, plan.chunk_off);
+                                                plan.seq_start, plan.chunk_off, plan.order);
     return cudaGetLastError();
 }
 

@@ -42,7 +42,7 @@ struct SimtParams {
     float scale;
     void *o;
     float *S_final;
-    const int32_t *seq_start, *chunk_off;
+    const int32_t *seq_start, *chunk_off, *order;
     float *ws;  // per-chunk intermediates
 };
 
@@ -181,7 +181,12 @@ __global__ void __launch_bounds__(kSimtThreads, 1) simt_carry_kernel(SimtParams 
     float *sS = sU + C * WV;     // [D][WV]  state slice
     float *sG = sS + D * WV;     // [D]
 
-    const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * WV, H = p.H;
+    // one CTA per (sequence, head, slice), sequences longest first
+    constexpr int kSlices = D / WV;
+    const int H = p.H;
+    const int j0 = (blockIdx.x % kSlices) * WV;
+    const int h = (blockIdx.x / kSlices) % H;
+    const int n = p.order[blockIdx.x / (kSlices * H)];
     const int tid = threadIdx.x, j = tid % WV, grp = tid / WV;  // 8 groups
     constexpr int NG = kSimtThreads / WV;
     const size_t sbase = ((size_t)n * H + h) * D * D;
@@ -267,7 +272,8 @@ cudaError_t launch_simt_d(const Problem &pb, void *workspace, int phases, cudaSt
     Plan plan;
     plan.seq_start = static_cast<int32_t *>(workspace);
     plan.chunk_off = plan.seq_start + (pb.N + 1);
-    p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off;
+    plan.order = plan.chunk_off + (pb.N + 1);
+    p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off; p.order = plan.order;
     p.ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + lay.plan_bytes);
 
     cudaError_t e;
@@ -287,7 +293,7 @@ cudaError_t launch_simt_d(const Problem &pb, void *workspace, int phases, cudaSt
         }
     }
     if (phases & kPhaseCarry) {
-        carry<<<dim3(pb.N, pb.H, D / kSimtSlice), kSimtThreads, carry_smem<D>(), st>>>(p);
+        carry<<<(unsigned)(pb.N * pb.H * (D / kSimtSlice)), kSimtThreads, carry_smem<D>(), st>>>(p);
         e = cudaGetLastError();
     }
     return e;
@@ -309,7 +315,7 @@ cudaError_t launch_simt_t(const Problem &p, void *ws, int ph, cudaStream_t st)
 WorkspaceLayout simt_workspace_layout(const Problem &p)
 {
     WorkspaceLayout l;
-    l.plan_bytes = align_up(sizeof(int32_t) * 2 * (size_t)(p.N + 1), 256);
+    l.plan_bytes = align_up(sizeof(int32_t) * plan_ints(p.N), 256);
     const size_t D = (size_t)p.dk;
     l.chunk_bytes = sizeof(float) * (4 * C * D + C * C + D) * (size_t)p.H * (size_t)p.max_chunks;
     l.total = l.plan_bytes + l.chunk_bytes;

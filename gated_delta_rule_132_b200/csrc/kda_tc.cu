@@ -76,7 +76,7 @@ struct TcParams {
     float scale;
     __nv_bfloat16 *o;
     float *S_final;
-    const int32_t *seq_start, *chunk_off;
+    const int32_t *seq_start, *chunk_off, *order;
     uint8_t *rec;      // records
     int *err;          // device error word (pipeline timeouts)
     int *fix_count;    // number of chunks listed for the exact fixup
@@ -255,15 +255,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Y = sum_k A[ai + rr][aj + k] * T[tj0 + k][tc0 + cc] over k in [0,16), for the
-// thread's (rr, cc); matrices in the [64][65] fp32 layout.
-__device__ __forceinline__ float blk_dot(const float *A, int ar, int ac, const float *T, int tr,
-                                         int tc, int rr, int cc)
+// sum_k X[xr + rr][xc + k] * Y[(yr + k) * ys + yc + cc] over k in [0,16): a 16-term
+// dot product of a row of X ([64][65] fp32) and a column of Y (row stride ys).
+// All 32 operands are loaded before the arithmetic and the sum runs in four
+// independent chains, so shared-memory latency is paid once, not per term.
+__device__ __forceinline__ float blk_dot(const float *X, int xr, int xc, const float *Y, int yr,
+                                         int yc, int ys, int rr, int cc)
 {
-    float acc = 0.f;
+    float a[16], b[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc += A[(ar + rr) * 65 + ac + k] * T[(tr + k) * 65 + tc + cc];
-    return acc;
+    for (int k = 0; k < 16; ++k) {
+        a[k] = X[(xr + rr) * 65 + xc + k];
+        b[k] = Y[(yr + k) * ys + yc + cc];
+    }
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+        s0 += a[k] * b[k]; s1 += a[k + 1] * b[k + 1];
+        s2 += a[k + 2] * b[k + 2]; s3 += a[k + 3] * b[k + 3];
+    }
+    return (s0 + s1) + (s2 + s3);
 }
 
 __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
@@ -529,17 +540,19 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         uint4 *z = reinterpret_cast<uint4 *>(sm + Prep2Smem::kTt + 8192);
         for (int i = tid; i < 8192 / 16; i += kPrep2Threads) z[i] = make_uint4(0, 0, 0, 0);
     }
-    if (tid < 64) {  // diagonal blocks: one column of one block per thread
+    if (tid < 64) {  // diagonal blocks: one column of one block per thread, right-looking
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            float acc = x[r];
+        for (int s2 = 0; s2 < 15; ++s2) {
+            float col[15];
 #pragma unroll
-            for (int s2 = 0; s2 < r; ++s2) acc -= As[(o + r) * 65 + o + s2] * x[s2];
-            x[r] = acc;
+            for (int r = s2 + 1; r < 16; ++r) col[r - 1] = As[(o + r) * 65 + o + s2];
+            const float xs = x[s2];
+#pragma unroll
+            for (int r = s2 + 1; r < 16; ++r) x[r] -= col[r - 1] * xs;
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Ts[(o + r) * 65 + o + cc] = x[r];
@@ -547,43 +560,39 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     __syncthreads();
     const int rr = tid >> 4, cc = tid & 15;
     // distance 1: T_{i,i-1} = -T_ii (A_{i,i-1} T_{i-1,i-1}), i = 1..3
-    for (int i = 1; i < 4; ++i)
-        Ys[(i - 1) * 256 + rr * 16 + cc] =
-            blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), rr, cc);
-    __syncthreads();
-    for (int i = 1; i < 4; ++i) {
-        float acc = 0.f;
+    float y[3];
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-            acc += Ts[(16 * i + rr) * 65 + 16 * i + k] * Ys[(i - 1) * 256 + k * 16 + cc];
-        Ts[(16 * i + rr) * 65 + 16 * (i - 1) + cc] = -acc;
-    }
+    for (int i = 1; i < 4; ++i)
+        y[i - 1] = blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), 65, rr, cc);
+#pragma unroll
+    for (int i = 1; i < 4; ++i) Ys[(i - 1) * 256 + rr * 16 + cc] = y[i - 1];
+    __syncthreads();
+#pragma unroll
+    for (int i = 1; i < 4; ++i)
+        y[i - 1] = -blk_dot(Ts, 16 * i, 16 * i, Ys + (i - 1) * 256, 0, 0, 16, rr, cc);
+#pragma unroll
+    for (int i = 1; i < 4; ++i) Ts[(16 * i + rr) * 65 + 16 * (i - 1) + cc] = y[i - 1];
     __syncthreads();
     // distance 2: T_{i,i-2} = -T_ii (A_{i,i-2} T_{i-2,i-2} + A_{i,i-1} T_{i-1,i-2}), i = 2, 3
-    for (int i = 2; i < 4; ++i)
-        Ys[(i - 2) * 256 + rr * 16 + cc] =
-            blk_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), rr, cc) +
-            blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), rr, cc);
-    __syncthreads();
-    for (int i = 2; i < 4; ++i) {
-        float acc = 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-            acc += Ts[(16 * i + rr) * 65 + 16 * i + k] * Ys[(i - 2) * 256 + k * 16 + cc];
-        Ts[(16 * i + rr) * 65 + 16 * (i - 2) + cc] = -acc;
-    }
+    for (int i = 2; i < 4; ++i)
+        y[i - 2] = blk_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), 65, rr, cc) +
+                   blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), 65, rr, cc);
+#pragma unroll
+    for (int i = 2; i < 4; ++i) Ys[(i - 2) * 256 + rr * 16 + cc] = y[i - 2];
+    __syncthreads();
+#pragma unroll
+    for (int i = 2; i < 4; ++i)
+        y[i - 2] = -blk_dot(Ts, 16 * i, 16 * i, Ys + (i - 2) * 256, 0, 0, 16, rr, cc);
+#pragma unroll
+    for (int i = 2; i < 4; ++i) Ts[(16 * i + rr) * 65 + 16 * (i - 2) + cc] = y[i - 2];
     __syncthreads();
     // distance 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)
-    Ys[rr * 16 + cc] = blk_dot(As, 48, 0, Ts, 0, 0, rr, cc) +
-                       blk_dot(As, 48, 16, Ts, 16, 0, rr, cc) +
-                       blk_dot(As, 48, 32, Ts, 32, 0, rr, cc);
+    Ys[rr * 16 + cc] = blk_dot(As, 48, 0, Ts, 0, 0, 65, rr, cc) +
+                       blk_dot(As, 48, 16, Ts, 16, 0, 65, rr, cc) +
+                       blk_dot(As, 48, 32, Ts, 32, 0, 65, rr, cc);
     __syncthreads();
-    {
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) acc += Ts[(48 + rr) * 65 + 48 + k] * Ys[k * 16 + cc];
-        Ts[(48 + rr) * 65 + cc] = -acc;
-    }
+    Ts[(48 + rr) * 65 + cc] = -blk_dot(Ts, 48, 48, Ys, 0, 0, 16, rr, cc);
     __syncthreads();
     {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
@@ -690,7 +699,11 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
     volatile int *abort = reinterpret_cast<volatile int *>(bars + 7);
 
-    const int n = blockIdx.x, h = blockIdx.y, half = blockIdx.z, H = p.H;
+    // one CTA per (sequence, head, half), sequences longest first
+    const int H = p.H;
+    const int half = blockIdx.x % kSlices;
+    const int h = (blockIdx.x / kSlices) % H;
+    const int n = p.order[blockIdx.x / (kSlices * H)];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -891,7 +904,7 @@ WorkspaceLayout tc_workspace_layout(const Problem &p)
 {
     WorkspaceLayout l;
     // plan arrays, the error word, the fixup count and the fixup list
-    l.plan_bytes = align_up(sizeof(int32_t) * (2 * (size_t)(p.N + 1) + 2 +
+    l.plan_bytes = align_up(sizeof(int32_t) * (plan_ints(p.N) + 2 +
                                                (size_t)p.max_chunks * p.H), 1024);
     l.chunk_bytes = (size_t)Record::kBytes * (size_t)p.H * (size_t)p.max_chunks;
     l.total = l.plan_bytes + l.chunk_bytes;
@@ -911,8 +924,9 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
     Plan plan;
     plan.seq_start = static_cast<int32_t *>(workspace);
     plan.chunk_off = plan.seq_start + (pb.N + 1);
-    p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off;
-    p.err = plan.chunk_off + (pb.N + 1);
+    plan.order = plan.chunk_off + (pb.N + 1);
+    p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off; p.order = plan.order;
+    p.err = plan.order + pb.N;
     p.fix_count = p.err + 1;
     p.fix_list = p.err + 2;
     p.rec = static_cast<uint8_t *>(workspace) + lay.plan_bytes;
@@ -942,7 +956,7 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
         e = cudaFuncSetAttribute(tc_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)CarrySmem::kBytes);
         if (e != cudaSuccess) return e;
-        tc_carry_kernel<<<dim3(pb.N, pb.H, kSlices), kCarryThreads, CarrySmem::kBytes, st>>>(p);
+        tc_carry_kernel<<<(unsigned)(pb.N * pb.H * kSlices), kCarryThreads, CarrySmem::kBytes, st>>>(p);
         e = cudaGetLastError();
     }
     return e;
