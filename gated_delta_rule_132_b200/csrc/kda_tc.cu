@@ -309,12 +309,31 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         *abort = 0;
         tc::fence_mbar_init();
     }
+    // Each thread copies the 16-byte granules it will read (its 8 channels of
+    // q, k, v and log_alpha for its 4 tokens) into the operand buffers, which
+    // step 1 fills only after every thread holds its inputs in registers: the
+    // chunk's 80 KB are in flight at once without holding registers.
+    uint8_t *in_q = sm + Prep2Smem::kAop, *in_k = sm + Prep2Smem::kAop + 16384;
+    uint8_t *in_v = sm + Prep2Smem::kBop, *in_la = sm + Prep2Smem::kBK;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int r = tg * 4 + e;
+        if (r < L) {
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
+            tc::cp_async16(in_q + r * 256 + oc * 16, p.q + off);
+            tc::cp_async16(in_k + r * 256 + oc * 16, p.k + off);
+            tc::cp_async16(in_v + r * 256 + oc * 16, p.v + off);
+            tc::cp_async16(in_la + r * 512 + oc * 32, p.log_alpha + off);
+            tc::cp_async16(in_la + r * 512 + oc * 32 + 16, p.log_alpha + off + 4);
+        }
+    }
     if (warp == 0) { tc::tmem_alloc(tmem_slot, 256); tc::tmem_relinquish(); }
     if (tid < C) sbeta[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * H + h] : 0.f;
 
     // ---- 1. loads and the cumulative log-decay
     uint4 qv[4], kv[4], vv[4];
     float g[4][8];
+    tc::cp_async_wait_all();
     {
         float run[8];
 #pragma unroll
@@ -325,12 +344,11 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
             uint4 q4 = make_uint4(0, 0, 0, 0), k4 = q4, v4 = q4;
             float4 la0 = make_float4(0.f, 0.f, 0.f, 0.f), la1 = la0;
             if (r < L) {
-                const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
-                q4 = __ldg(reinterpret_cast<const uint4 *>(p.q + off));
-                k4 = __ldg(reinterpret_cast<const uint4 *>(p.k + off));
-                v4 = __ldg(reinterpret_cast<const uint4 *>(p.v + off));
-                la0 = __ldg(reinterpret_cast<const float4 *>(p.log_alpha + off));
-                la1 = __ldg(reinterpret_cast<const float4 *>(p.log_alpha + off + 4));
+                q4 = *reinterpret_cast<const uint4 *>(in_q + r * 256 + oc * 16);
+                k4 = *reinterpret_cast<const uint4 *>(in_k + r * 256 + oc * 16);
+                v4 = *reinterpret_cast<const uint4 *>(in_v + r * 256 + oc * 16);
+                la0 = *reinterpret_cast<const float4 *>(in_la + r * 512 + oc * 32);
+                la1 = *reinterpret_cast<const float4 *>(in_la + r * 512 + oc * 32 + 16);
             }
             qv[e] = q4; kv[e] = k4; vv[e] = v4;
             run[0] += la0.x; run[1] += la0.y; run[2] += la0.z; run[3] += la0.w;
