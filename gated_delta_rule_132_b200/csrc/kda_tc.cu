@@ -233,10 +233,10 @@ constexpr int kPrep2Threads = 256;
 
 struct Prep2Smem {
     static constexpr uint32_t kAop = 0;        // 32768: [kb][128 rows][128B]
-    static constexpr uint32_t kA = 0;          // fp32 A [64][65], after MMA-AP
+    static constexpr uint32_t kA = 0;          // fp32 A [64][kLd], after MMA-AP
     static constexpr uint32_t kBop = 32768;    // 24576: [kb][96 rows][128B]
-    static constexpr uint32_t kT = 32768;      // fp32 T [64][65], after MMA-AP
-    static constexpr uint32_t kY = 49408;      // fp32 3 x [16][16] block products
+    static constexpr uint32_t kT = 32768;      // fp32 T [64][kLd], after MMA-AP
+    static constexpr uint32_t kY = 50176;      // fp32 3 x [16][16] block products
     static constexpr uint32_t kBK = 57344;     // 16384: (beta K~) MN-major image
     static constexpr uint32_t kBV = 73728;     // 16384: (beta V) MN-major image (follows BK)
     static constexpr uint32_t kTt = 90112;     // 16384: [T; 0], K-major rows r
@@ -255,27 +255,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// sum_k X[xr + rr][xc + k] * Y[(yr + k) * ys + yc + cc] over k in [0,16): a 16-term
-// dot product of a row of X ([64][65] fp32) and a column of Y (row stride ys).
-// All 32 operands are loaded before the arithmetic and the sum runs in four
-// independent chains, so shared-memory latency is paid once, not per term.
-__device__ __forceinline__ float blk_dot(const float *X, int xr, int xc, const float *Y, int yr,
-                                         int yc, int ys, int rr, int cc)
+// Row stride (floats) of the fp32 A and T matrices: rows stay 16-byte aligned,
+// and float4 stores of 8 consecutive rows hit distinct bank groups.
+constexpr int kLd = 68;
+
+// One 1x4 strip of a 16x16 block product:
+//     acc[q] += sum_k X[xr + rr][xc + k] * Y[yr + k][yc + 4*c4 + q],  k < 16, q < 4,
+// X with row stride kLd, Y with row stride ys. 4 + 16 vector loads feed 64 FMAs
+// in four independent chains.
+__device__ __forceinline__ void strip_dot(const float *X, int xr, int xc, const float *Y, int yr,
+                                          int yc, int ys, int rr, int c4, float4 &acc)
 {
-    float a[16], b[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        a[k] = X[(xr + rr) * 65 + xc + k];
-        b[k] = Y[(yr + k) * ys + yc + cc];
-    }
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    float a[16];
 #pragma unroll
     for (int k = 0; k < 16; k += 4) {
-        s0 += a[k] * b[k]; s1 += a[k + 1] * b[k + 1];
-        s2 += a[k + 2] * b[k + 2]; s3 += a[k + 3] * b[k + 3];
+        const float4 v = *reinterpret_cast<const float4 *>(X + (xr + rr) * kLd + xc + k);
+        a[k] = v.x; a[k + 1] = v.y; a[k + 2] = v.z; a[k + 3] = v.w;
     }
-    return (s0 + s1) + (s2 + s3);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float4 y = *reinterpret_cast<const float4 *>(Y + (yr + k) * ys + yc + 4 * c4);
+        acc.x += a[k] * y.x; acc.y += a[k] * y.y; acc.z += a[k] * y.z; acc.w += a[k] * y.w;
+    }
 }
+
+__device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y, -v.z, -v.w); }
 
 __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
 {
@@ -510,8 +514,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         }
         tc::mma_commit(bar_ap);
     }
-    float *As = reinterpret_cast<float *>(sm + Prep2Smem::kA);   // A[r][s], stride 65
-    float *Ts = reinterpret_cast<float *>(sm + Prep2Smem::kT);   // T[r][s], stride 65
+    float *As = reinterpret_cast<float *>(sm + Prep2Smem::kA);   // A[r][s], stride kLd
+    float *Ts = reinterpret_cast<float *>(sm + Prep2Smem::kT);   // T[r][s], stride kLd
     float *Ys = reinterpret_cast<float *>(sm + Prep2Smem::kY);
     {
         // every warp reads its 32 TMEM lanes; warps 0-3 take the first 32 of the
@@ -529,9 +533,14 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         if (is_k) {
             const float b = sbeta[r];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int s2 = sh + e;
-                As[r * 65 + s2] = (s2 < lim && s2 < r) ? b * d[e] : 0.f;
+            for (int e = 0; e < 32; e += 4) {
+                float v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int s2 = sh + e + q;
+                    v[q] = (s2 < lim && s2 < r) ? b * d[e + q] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(As + r * kLd + sh + e) = make_float4(v[0], v[1], v[2], v[3]);
             }
         } else {
             uint8_t *prow = rec + Record::kP;
@@ -567,50 +576,63 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         for (int s2 = 0; s2 < 15; ++s2) {
             float col[15];
 #pragma unroll
-            for (int r = s2 + 1; r < 16; ++r) col[r - 1] = As[(o + r) * 65 + o + s2];
+            for (int r = s2 + 1; r < 16; ++r) col[r - 1] = As[(o + r) * kLd + o + s2];
             const float xs = x[s2];
 #pragma unroll
             for (int r = s2 + 1; r < 16; ++r) x[r] -= col[r - 1] * xs;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Ts[(o + r) * 65 + o + cc] = x[r];
+        for (int r = 0; r < 16; ++r) Ts[(o + r) * kLd + o + cc] = x[r];
     }
     __syncthreads();
-    const int rr = tid >> 4, cc = tid & 15;
-    // distance 1: T_{i,i-1} = -T_ii (A_{i,i-1} T_{i-1,i-1}), i = 1..3
-    float y[3];
-#pragma unroll
-    for (int i = 1; i < 4; ++i)
-        y[i - 1] = blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), 65, rr, cc);
-#pragma unroll
-    for (int i = 1; i < 4; ++i) Ys[(i - 1) * 256 + rr * 16 + cc] = y[i - 1];
+    // Off-diagonal blocks by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, in
+    // 1x4 strips: thread -> (block, row rr, column group c4).
+    const int rr = (tid & 63) >> 2, c4 = tid & 3, blk = tid >> 6;
+    // distance 1: i = 1..3 on threads 0..191
+    if (blk < 3) {
+        const int i = 1 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), kLd, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ys + blk * 256 + rr * 16 + 4 * c4) = acc;
+    }
     __syncthreads();
-#pragma unroll
-    for (int i = 1; i < 4; ++i)
-        y[i - 1] = -blk_dot(Ts, 16 * i, 16 * i, Ys + (i - 1) * 256, 0, 0, 16, rr, cc);
-#pragma unroll
-    for (int i = 1; i < 4; ++i) Ts[(16 * i + rr) * 65 + 16 * (i - 1) + cc] = y[i - 1];
+    if (blk < 3) {
+        const int i = 1 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(Ts, 16 * i, 16 * i, Ys + blk * 256, 0, 0, 16, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ts + (16 * i + rr) * kLd + 16 * (i - 1) + 4 * c4) = neg4(acc);
+    }
     __syncthreads();
-    // distance 2: T_{i,i-2} = -T_ii (A_{i,i-2} T_{i-2,i-2} + A_{i,i-1} T_{i-1,i-2}), i = 2, 3
-#pragma unroll
-    for (int i = 2; i < 4; ++i)
-        y[i - 2] = blk_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), 65, rr, cc) +
-                   blk_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), 65, rr, cc);
-#pragma unroll
-    for (int i = 2; i < 4; ++i) Ys[(i - 2) * 256 + rr * 16 + cc] = y[i - 2];
+    // distance 2: i = 2, 3 on threads 0..127
+    if (blk < 2) {
+        const int i = 2 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), kLd, rr, c4, acc);
+        strip_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), kLd, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ys + blk * 256 + rr * 16 + 4 * c4) = acc;
+    }
     __syncthreads();
-#pragma unroll
-    for (int i = 2; i < 4; ++i)
-        y[i - 2] = -blk_dot(Ts, 16 * i, 16 * i, Ys + (i - 2) * 256, 0, 0, 16, rr, cc);
-#pragma unroll
-    for (int i = 2; i < 4; ++i) Ts[(16 * i + rr) * 65 + 16 * (i - 2) + cc] = y[i - 2];
+    if (blk < 2) {
+        const int i = 2 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(Ts, 16 * i, 16 * i, Ys + blk * 256, 0, 0, 16, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ts + (16 * i + rr) * kLd + 16 * (i - 2) + 4 * c4) = neg4(acc);
+    }
     __syncthreads();
-    // distance 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20)
-    Ys[rr * 16 + cc] = blk_dot(As, 48, 0, Ts, 0, 0, 65, rr, cc) +
-                       blk_dot(As, 48, 16, Ts, 16, 0, 65, rr, cc) +
-                       blk_dot(As, 48, 32, Ts, 32, 0, 65, rr, cc);
+    // distance 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20) on threads 0..63
+    if (blk == 0) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(As, 48, 0, Ts, 0, 0, kLd, rr, c4, acc);
+        strip_dot(As, 48, 16, Ts, 16, 0, kLd, rr, c4, acc);
+        strip_dot(As, 48, 32, Ts, 32, 0, kLd, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ys + rr * 16 + 4 * c4) = acc;
+    }
     __syncthreads();
-    Ts[(48 + rr) * 65 + cc] = -blk_dot(Ts, 48, 48, Ys, 0, 0, 16, rr, cc);
+    if (blk == 0) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(Ts, 48, 48, Ys, 0, 0, 16, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ts + (48 + rr) * kLd + 4 * c4) = neg4(acc);
+    }
     __syncthreads();
     {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
@@ -621,8 +643,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int sa = s0 + h2 * 8 + 2 * e, sb2 = sa + 1;
-                const float va = sa < r ? Ts[r * 65 + sa] : (sa == r ? 1.f : 0.f);
-                const float vb = sb2 < r ? Ts[r * 65 + sb2] : (sb2 == r ? 1.f : 0.f);
+                const float va = sa < r ? Ts[r * kLd + sa] : (sa == r ? 1.f : 0.f);
+                const float vb = sb2 < r ? Ts[r * kLd + sb2] : (sb2 == r ? 1.f : 0.f);
                 w[e] = pack_bf16x2(va, vb);
             }
             *reinterpret_cast<uint4 *>(tt + tc::sw128(r, (s0 + h2 * 8) * 2)) =
