@@ -415,81 +415,95 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w; a[4] = y.x; a[5] = y.y; a[6] = y.z; a[7] = y.w;
     };
     const bool first_half = tg < 8;
+    // Products that only feed bf16 operands are formed in packed bf16 (two per
+    // instruction): the factor is rounded to bf16 once, the product once more.
+    auto to2 = [](const float *a, __nv_bfloat162 *b2) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b2[j] = __floats2bfloat162_rn(a[2 * j], a[2 * j + 1]);
+    };
+    auto mul4 = [](const uint4 &x, const __nv_bfloat162 *f) {
+        const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
+        uint4 r;
+        __nv_bfloat162 *r2 = reinterpret_cast<__nv_bfloat162 *>(&r);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r2[j] = __hmul2(x2[j], f[j]);
+        return r;
+    };
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int r = tg * 4 + e;
         const uint32_t sw = ((ck ^ (uint32_t)(r & 7)) << 4);  // swizzled chunk offset
         const float *ge = g[e];
         const uint4 qe = qv[e], ke = kv[e], ve = vv[e];
-        float qf[8], kf[8], E[8], Hh[8], o[8];
-        unpack8(qe, qf); unpack8(ke, kf);
-        ld8(2, o);  // gC
+        float E[8], Hh[8], t8[8];
+        __nv_bfloat162 f2[4];
+        ld8(2, t8);  // g_C
 #pragma unroll
-        for (int j = 0; j < 8; ++j) { E[j] = __expf(ge[j]); Hh[j] = __expf(o[j] - ge[j]); }
+        for (int j = 0; j < 8; ++j) { E[j] = __expf(ge[j]); Hh[j] = __expf(t8[j] - ge[j]); }
         const float b = sbeta[r];
         // record: Q~ (rows 64.. of A1) and K^ (MN-major image)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] = qf[j] * E[j];
-        *reinterpret_cast<uint4 *>(rec + Record::kA1 + kb * 16384 + (64 + r) * 128 + sw) = pack8(o);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] = kf[j] * Hh[j];
-        *reinterpret_cast<uint4 *>(rec + Record::kKh + kb * 8192 + r * 128 + sw) = pack8(o);
+        to2(E, f2);
+        *reinterpret_cast<uint4 *>(rec + Record::kA1 + kb * 16384 + (64 + r) * 128 + sw) = mul4(qe, f2);
+        to2(Hh, f2);
+        *reinterpret_cast<uint4 *>(rec + Record::kKh + kb * 8192 + r * 128 + sw) = mul4(ke, f2);
         // solve right-hand sides (MN-major: token rows, channel columns)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] = b * kf[j] * E[j];
-        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBK + kb * 8192 + r * 128 + sw) = pack8(o);
-        unpack8(ve, o);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] *= b;
-        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBV + kb * 8192 + r * 128 + sw) = pack8(o);
-        // factors for the A/P contraction: row factor -> E (in place), column
-        // factors -> Hh (in place) and o
+        for (int j = 0; j < 8; ++j) t8[j] = b * E[j];
+        to2(t8, f2);
+        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBK + kb * 8192 + r * 128 + sw) = mul4(ke, f2);
+        {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(b, b);
+            const __nv_bfloat162 bb[4] = {b2, b2, b2, b2};
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBV + kb * 8192 + r * 128 + sw) = mul4(ve, bb);
+        }
+        // factors for the A/P contraction: row factor (k and q rows) and the
+        // column factor(s) (k rows of the B operand)
         float ref[8];
         if (first_half) {
+            float c0f[8], c1f[8];
             if (fast) {
                 ld8(3, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) E[j] *= ref[j];          // e^{g_r - g_15}
-                ld8(6, ref);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = Hh[j] * ref[j];   // e^{g_31 - g_r}
+                for (int j = 0; j < 8; ++j) E[j] *= ref[j];            // e^{g_r - g_15}
                 ld8(5, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) Hh[j] *= ref[j];         // e^{g_15 - g_r}
+                for (int j = 0; j < 8; ++j) c0f[j] = Hh[j] * ref[j];   // e^{g_15 - g_r}
+                ld8(6, ref);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) c1f[j] = Hh[j] * ref[j];   // e^{g_31 - g_r}
             } else {
                 ld8(0, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) { E[j] = cexp(ge[j] - ref[j]); Hh[j] = cexp(ref[j] - ge[j]); }
+                for (int j = 0; j < 8; ++j) { E[j] = cexp(ge[j] - ref[j]); c0f[j] = cexp(ref[j] - ge[j]); }
                 ld8(1, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = cexp(ref[j] - ge[j]);
+                for (int j = 0; j < 8; ++j) c1f[j] = cexp(ref[j] - ge[j]);
             }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { Hh[j] *= kf[j]; o[j] *= kf[j]; }
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + r * 128 + sw) = pack8(Hh);
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + (32 + r) * 128 + sw) = pack8(o);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { o[j] = kf[j] * E[j]; qf[j] *= E[j]; }
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + r * 128 + sw) = pack8(o);
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = pack8(qf);
+            to2(c0f, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + r * 128 + sw) = mul4(ke, f2);
+            to2(c1f, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + (32 + r) * 128 + sw) = mul4(ke, f2);
+            to2(E, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + r * 128 + sw) = mul4(ke, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = mul4(qe, f2);
         } else {
             if (fast) {
                 ld8(4, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) E[j] *= ref[j];          // e^{g_r - g_31}
+                for (int j = 0; j < 8; ++j) E[j] *= ref[j];            // e^{g_r - g_31}
                 ld8(6, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) Hh[j] *= ref[j];         // e^{g_31 - g_r}
+                for (int j = 0; j < 8; ++j) Hh[j] *= ref[j];           // e^{g_31 - g_r}
             } else {
                 ld8(1, ref);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) { E[j] = cexp(ge[j] - ref[j]); Hh[j] = cexp(ref[j] - ge[j]); }
             }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { Hh[j] *= kf[j]; o[j] = kf[j] * E[j]; qf[j] *= E[j]; }
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + (32 + r) * 128 + sw) = pack8(Hh);
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = pack8(o);
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (64 + r) * 128 + sw) = pack8(qf);
+            to2(Hh, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBop + kb * 12288 + (32 + r) * 128 + sw) = mul4(ke, f2);
+            to2(E, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = mul4(ke, f2);
+            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (64 + r) * 128 + sw) = mul4(qe, f2);
         }
     }
     // A chunk whose decay inside half a chunk exceeds the factorised range is
