@@ -725,11 +725,12 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
 // Warps 0-7 (256 threads) own the 128 x 64 state slice: warp w serves TMEM lanes
 // 32*(w%4).. (state rows) and value columns 32*(w/4).. of the slice, so each
 // thread keeps one state row x 32 columns in fp32 registers. Warp 8 streams
-// records. Thread 0 issues each MMA group right after the named barrier that
-// completes its operands, so the waits on the critical path are the two MMA
-// completions per chunk plus the epilogues. The output accumulator D1 is
-// double-buffered in TMEM, so the output rows of chunk c are read (warps
-// serving lanes 64..127) after chunk c+1's first MMA group is already issued.
+// records. Thread 0 issues the two state MMA groups right after the named
+// barrier that completes their operands; lane 1 of warp 8 issues the
+// output-only product [0;P] U right behind K^^T U, so the state update does
+// not wait for it. The output accumulator D1 is double-buffered in TMEM, so the
+// output rows of chunk c are read (warps serving lanes 64..127) after chunk
+// c+1's first MMA group is already issued.
 constexpr int kCarryThreads = 288;
 constexpr uint32_t kTmemCols = 256;  // D1[0]: [0,64), D2: [64,128), D1[1]: [128,192)
 
@@ -750,8 +751,10 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     uint64_t *empty = bars + 2;  // [2]
     uint64_t *d1_done = bars + 4;
     uint64_t *d2_done = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 7);
+    uint64_t *pu_go = bars + 6;    // K^^T U issued: the [0;P] U group may follow
+    uint64_t *pu_done = bars + 7;  // [0;P] U completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 9);
 
     // one CTA per (sequence, head, half), sequences longest first
     const int H = p.H;
@@ -764,6 +767,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         tc::mbar_init(&full[0], 1); tc::mbar_init(&full[1], 1);
         tc::mbar_init(&empty[0], 8); tc::mbar_init(&empty[1], 8);
         tc::mbar_init(d1_done, 1); tc::mbar_init(d2_done, 1);
+        tc::mbar_init(pu_go, 1); tc::mbar_init(pu_done, 1);
         *abort = 0;
         tc::fence_mbar_init();
     }
@@ -800,6 +804,22 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             // every issued copy has landed before the CTA may exit
             for (int lc = (nc > 2 ? nc - 2 : 0); lc < nc; ++lc)
                 tc::mbar_wait(&full[lc & 1], (lc >> 1) & 1, abort, p.err, kErrFull);
+        } else if (lane == 1) {
+            // The output-only product [0; P] U: queued right behind K^^T U, so the
+            // state update (which waits only for K^^T U) does not wait for it.
+            const uint32_t id2b = tc::idesc_bf16(128, 64, 0, 1);
+            const uint32_t b2 = tc::smem_u32(sm + CarrySmem::kB2);
+            for (int lc = 0; lc < nc; ++lc) {
+                const int st = lc & 1;
+                tc::mbar_wait(pu_go, lc & 1, abort, p.err, kErrD2);
+                tc::tc_fence_after_sync();
+                const uint32_t a2b = tc::smem_u32(sm + st * CarrySmem::kStage + CarrySmem::kA2b);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + (uint32_t)st * 128, tc::smem_desc(a2b + kk * 32, 16, 1024),
+                                 tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2b, 1);
+                tc::mma_commit(pu_done);
+            }
         }
     } else {
         // ---------------- state owners
@@ -809,7 +829,6 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         const uint32_t lane_addr = tmem + ((uint32_t)(lg * 32) << 16);
         const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 1);   // [W;Q~] K-major . S MN-major
         const uint32_t id2a = tc::idesc_bf16(128, 64, 1, 1);  // K^^T MN-major . U MN-major
-        const uint32_t id2b = tc::idesc_bf16(128, 64, 0, 1);  // [0;P] K-major . U MN-major
         const uint32_t b1 = tc::smem_u32(sm + CarrySmem::kB1);
         const uint32_t b2 = tc::smem_u32(sm + CarrySmem::kB2);
         float S[32];
@@ -900,16 +919,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
                 if (threadIdx.x == 0) {
                     tc::tc_fence_after_sync();
                     const uint32_t kh = tc::smem_u32(sb + CarrySmem::kKh);
-                    const uint32_t a2b = tc::smem_u32(sb + CarrySmem::kA2b);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma_bf16(tmem + 64, tc::smem_desc(kh + kk * 2048, 8192, 1024),
                                      tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2a, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(d1, tc::smem_desc(a2b + kk * 32, 16, 1024),
-                                     tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2b, 1);
                     tc::mma_commit(d2_done);
+                    tc::mbar_arrive(pu_go);
                 }
             }
             // D. S = gamma * S + K^^T U, and its bf16 copy for the next MMA1
@@ -925,6 +940,11 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             store_bf16(sm + CarrySmem::kB1, t, S);
             tc::fence_proxy_async_smem();
             tc::tc_fence_before_sync();
+            // [0;P] U (another thread's commit) has finished reading this stage and
+            // B2 and adding into D1[st]: the stage can go back to the producer, the
+            // next chunk may rewrite B2 and write_o may read D1[st]
+            tc::mbar_wait(pu_done, lc & 1, abort, p.err, kErrD2);
+            tc::tc_fence_after_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&empty[st]);
         }
