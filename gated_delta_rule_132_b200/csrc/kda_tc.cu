@@ -16,15 +16,15 @@
 //    gamma and U~. One record per (chunk, head), see Record below.
 //  * carry (sequential, one CTA per sequence, head and 64-column half of the
 //    value dimension; the value columns of S never mix) walks the chunks in
-//    order. Warp 4 streams each record into a two-stage shared-memory ring
-//    with bulk async copies; warp 5 issues the tcgen05 MMAs; warps 0-3 own the
-//    128 rows of the state slice (fp32, in registers), read the accumulators
-//    out of TMEM and write the bf16 operands the next MMA needs:
-//        MMA1: D1 = [W; Q~] (128x128) . S (128x64)        -> WS rows, Q~S rows
-//        U    = U~ - WS                                    (warps 0-1)
-//        MMA2: D2 = K^^T (128x64) . U (64x64)              -> state increment
-//              D1 += [0; P] (128x64) . U                   -> Q~S + PU
-//        S    = gamma * S + D2 (warps 0-3); o = scale * D1 rows 64..127 (warps 2-3)
+//    order. Warp 8 streams each record into a two-stage shared-memory ring
+//    with bulk async copies; warp 9 issues the tcgen05 MMAs; warps 0-7 own the
+//    transposed state slice S^T (fp32, in registers), read the accumulators out
+//    of TMEM and write the bf16 operands the next MMA needs:
+//        MMA1: D1 = S^T . [W; Q~]^T            -> (W S)^T | (Q~ S)^T
+//        U^T  = U~^T - (W S)^T
+//        MMA2: D2 = U^T . K^                    -> state increment (K^^T U)^T
+//        MMA3: D1[:, 64:] += U^T . P^T          -> (Q~ S + P U)^T
+//        S^T  = S^T Diag(gamma) + D2;  o = scale * D1[:, 64:]^T
 //    The state never leaves the SM between chunks; S_final is written once.
 #include "kda_internal.cuh"
 #include "tc_primitives.cuh"
@@ -44,28 +44,31 @@ struct Record {
     static constexpr uint32_t kKh = 32768;    // K^^T 128x64 bf16, MN-major, SW128, 2 MN-blocks
     static constexpr uint32_t kP = 49152;     // P 64x64 bf16, K-major, SW128
     static constexpr uint32_t kG = 57344;     // gamma fp32 [128]
-    static constexpr uint32_t kU = 57856;     // U~ fp32 [2 halves][64 rows][64 cols], 16B-chunk swizzled
+    static constexpr uint32_t kU = 57856;     // U~^T fp32 [2 halves][64 value cols][64 tokens], 16B-chunk swizzled
     static constexpr uint32_t kBytes = 90624;
 };
 static_assert(Record::kU + kSlices * C * kSlice * 4 == Record::kBytes, "record size");
 
 // Shared-memory layout of the carry kernel (offsets from a 1024-aligned base).
 struct CarrySmem {
-    static constexpr uint32_t kA1 = 0;         // 32768
-    static constexpr uint32_t kKh = 32768;     // 16384
-    static constexpr uint32_t kA2b = 49152;    // 16384: rows 0..63 zero, rows 64..127 = P
-    static constexpr uint32_t kU = 65536;      // 16384
-    static constexpr uint32_t kG = 81920;      // 512
-    static constexpr uint32_t kStage = 83968;  // stage stride (1024-aligned)
-    static constexpr uint32_t kB1 = 2 * kStage;        // S (bf16, 128x64, MN-major)
-    static constexpr uint32_t kB2 = kB1 + 16384;       // U (bf16, 64x64, MN-major)
-    static constexpr uint32_t kBar = kB2 + 8192;       // mbarriers
+    static constexpr uint32_t kA1 = 0;         // 32768: [W; Q~], B of MMA1 (K-major)
+    static constexpr uint32_t kKh = 32768;     // 16384: K^, B of MMA2 (MN-major)
+    static constexpr uint32_t kP = 49152;      // 8192:  P, B of MMA3 (K-major)
+    static constexpr uint32_t kU = 57344;      // 16384: U~^T of this half, fp32
+    static constexpr uint32_t kG = 73728;      // 512:   gamma
+    static constexpr uint32_t kStage = 74752;  // stage stride (1024-aligned)
+    static constexpr uint32_t kSt = 2 * kStage;        // S^T bf16 64x128, A of MMA1 (K-major, 2 K-blocks)
+    static constexpr uint32_t kUt = kSt + 16384;       // U^T bf16 64x64, A of MMA2/MMA3 (K-major)
+    static constexpr uint32_t kOs = kUt + 8192;        // output staging, 1 KB per state warp
+    static constexpr uint32_t kBar = kOs + 8192;       // mbarriers
     static constexpr uint32_t kBytes = kBar + 256 + 1024;  // + alignment slack
 };
+static_assert(CarrySmem::kSt % 1024 == 0 && CarrySmem::kUt % 1024 == 0, "operand alignment");
 
 __device__ __forceinline__ uint32_t u_swz(uint32_t r, uint32_t jj)
 {
-    // byte offset of U~[r][jj] inside one 64x64 fp32 half: 16-byte chunks XORed by row
+    // byte offset of element [r][jj] of a 64x64 fp32 tile (rows of 256 bytes):
+    // 16-byte chunks XORed by row
     return r * 256u + ((((jj >> 2) ^ (r & 15u)) << 4) | ((jj & 3u) << 2));
 }
 
@@ -193,7 +196,7 @@ __device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
         const uint32_t kb = (uint32_t)(i >> 6) * 16384u;
         a1[(kb + tc::sw128(r, 2 * (i & 63))) / 2] = __float2bfloat16_rn(sk[r * DP + i]);
         const int half = i >> 6, jj = i & 63;
-        *reinterpret_cast<float *>(uu + half * 16384 + u_swz(r, jj)) = sv[r * D + i];
+        *reinterpret_cast<float *>(uu + half * 16384 + u_swz(jj, r)) = sv[r * D + i];
     }
     __syncthreads();  // the caller reuses shared memory for its next chunk
 }
@@ -226,8 +229,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams
 //  3. T = (I + A)^{-1} in fp32 by blocks of 16: the four diagonal blocks by
 //     substitution, then the off-diagonal blocks by distance,
 //     T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, as 16x16 products on all threads.
-//  4. [W | U~] = [T; 0] (128x64) . [beta K~ | beta V] (64x256) as one MMA; rows
-//     0..63 of the accumulator are the 64 tokens.
+//  4. W = [T; 0] (128x64) . beta K~ (64x128), whose accumulator rows 0..63 are
+//     the 64 tokens, and U~^T = (beta V)^T (128x64) . T^T (64x64), whose rows
+//     are the 128 value columns: two MMA groups on the same operand images.
 //  5. Everything goes to the record in the carry kernel's operand layouts.
 constexpr int kPrep2Threads = 256;
 
@@ -400,15 +404,6 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     }
     bool clamped = false;
     auto cexp = [&](float x) { if (x > 80.f) { clamped = true; x = 80.f; } return __expf(x); };
-    auto pack8 = [](const float *a) {
-        return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]),
-                          pack_bf16x2(a[4], a[5]), pack_bf16x2(a[6], a[7]));
-    };
-    auto unpack8 = [](const uint4 &u, float *a) {
-        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) { a[2 * j] = __low2float(b[j]); a[2 * j + 1] = __high2float(b[j]); }
-    };
     auto ld8 = [&](int row, float *a) {  // 8 per-channel constants of this octet
         const float4 x = *reinterpret_cast<const float4 *>(cst + row * D + c0);
         const float4 y = *reinterpret_cast<const float4 *>(cst + row * D + c0 + 4);
@@ -670,48 +665,53 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     __syncthreads();
     tc::tc_fence_after_sync();
 
-    // ---- 4. [W | U~] = [T; 0] . [beta K~ | beta V]
+    // ---- 4. W = [T; 0] . beta K~ and U~^T = (beta V)^T . T^T
     if (tid == 0) {
-        const uint32_t bkv = tc::smem_u32(sm + Prep2Smem::kBK);  // 4 MN atoms: BK then BV
+        const uint32_t bk = tc::smem_u32(sm + Prep2Smem::kBK);  // 2 MN atoms (channels)
+        const uint32_t bv = tc::smem_u32(sm + Prep2Smem::kBV);
         const uint32_t tt = tc::smem_u32(sm + Prep2Smem::kTt);
-        const uint32_t id = tc::idesc_bf16(128, 256, 0, 1);
+        const uint32_t idw = tc::idesc_bf16(128, 128, 0, 1);  // rows: tokens (64 used)
+        const uint32_t idu = tc::idesc_bf16(128, 64, 1, 0);   // rows: value columns
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
             tc::mma_bf16(tmem, tc::smem_desc(tt + kk * 32, 16, 1024),
-                         tc::smem_desc(bkv + kk * 2048, 8192, 1024), id, kk > 0);
+                         tc::smem_desc(bk + kk * 2048, 8192, 1024), idw, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem + 128, tc::smem_desc(bv + kk * 2048, 8192, 1024),
+                         tc::smem_desc(tt + kk * 32, 16, 1024), idu, kk > 0);
         tc::mma_commit(bar_wu);
     }
-    if ((warp & 3) < 2) {  // warps 0,1: W (columns 0..127); warps 4,5: U~ (128..255)
+    {
+        // W: lanes 0..63 (tokens), columns 0..127 (channels 64*wh..): warps 0,1,4,5.
+        // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
         tc::mbar_wait(bar_wu, 0, abort, p.err, 12);
         tc::tc_fence_after_sync();
-        const int r = (warp & 3) * 32 + (tid & 31);  // token
-        const uint32_t la = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const int lg = warp & 3, wh = warp >> 2;
+        const int row = lg * 32 + (tid & 31);
+        const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
         float w[32];
-        if (warp < 4) {
+        if (lg < 2) {
+            uint8_t *a1 = rec + Record::kA1 + (uint32_t)wh * 16384;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                tc::tmem_ld32_sync(la + q4 * 32, w);
-                uint8_t *a1 = rec + Record::kA1 + (uint32_t)(q4 >> 1) * 16384;
+            for (int q2 = 0; q2 < 2; ++q2) {
+                tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
 #pragma unroll
                 for (int c16 = 0; c16 < 4; ++c16) {
                     uint32_t u[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
-                    *reinterpret_cast<uint4 *>(a1 + tc::sw128(r, ((q4 & 1) * 4 + c16) * 16)) =
+                    *reinterpret_cast<uint4 *>(a1 + tc::sw128(row, (q2 * 4 + c16) * 16)) =
                         make_uint4(u[0], u[1], u[2], u[3]);
                 }
             }
-        } else {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                tc::tmem_ld32_sync(la + 128 + q4 * 32, w);
-                uint8_t *uu = rec + Record::kU + (uint32_t)(q4 >> 1) * 16384;
-#pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    *reinterpret_cast<float4 *>(uu + u_swz(r, (q4 & 1) * 32 + 4 * m)) =
-                        make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
-            }
         }
+        tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
+        uint8_t *uu = rec + Record::kU + (uint32_t)(row >> 6) * 16384;
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            *reinterpret_cast<float4 *>(uu + u_swz(row & 63, 32 * wh + 4 * m)) =
+                make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
     }
     tc::tc_fence_before_sync();
     __syncthreads();
@@ -722,19 +722,33 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
 }
 
 // ------------------------------------------------------------------- carry
-// Warps 0-7 (256 threads) own the 128 x 64 state slice: warp w serves TMEM lanes
-// 32*(w%4).. (state rows) and value columns 32*(w/4).. of the slice, so each
-// thread keeps one state row x 32 columns in fp32 registers. Warp 8 streams
-// records. Thread 0 issues the two state MMA groups right after the named
-// barrier that completes their operands; lane 1 of warp 8 issues the
-// output-only product [0;P] U right behind K^^T U, so the state update does
-// not wait for it. The output accumulator D1 is double-buffered in TMEM, so the
-// output rows of chunk c are read (warps serving lanes 64..127) after chunk
-// c+1's first MMA group is already issued.
-constexpr int kCarryThreads = 288;
-constexpr uint32_t kTmemCols = 256;  // D1[0]: [0,64), D2: [64,128), D1[1]: [128,192)
+// The state slice is carried transposed, S^T (64 value columns x 128 key
+// channels), so that every product of a chunk step has the slice's 64 value
+// columns on the M side, and the 64 tokens of W and of Q~ share one N = 128:
+//     MMA1  D1       = S^T . [W; Q~]^T  (64x128, K = 128)  -> (W S)^T | (Q~ S)^T
+//     MMA2  D2       = U^T . K^         (64x128, K = 64)   -> (K^^T U)^T
+//     MMA3  D1[:,64:] += U^T . P^T      (64x64,  K = 64)   -> O^T = (Q~ S + P U)^T
+// with U^T = U~^T - (W S)^T and S^T <- S^T Diag(gamma) + D2. M = 64 products
+// issue in about two thirds of the time of M = 128 ones.
+// An M = 64 accumulator keeps row m in TMEM lane 32*(m/16) + m%16; warp w reads
+// rows 16*(w%4) .. +15 with the 16x32bx2 shape, lanes 0-15 and 16-31 splitting
+// the columns. Warps 0-7 own the state: thread (w, l) keeps S^T row
+// 16*(w%4) + l%16, key channels 64*(w/4) + 32*(l/16) .. +31, in fp32 registers.
+// Warp 8 streams the records into a two-stage ring with bulk copies. Warp 9
+// issues the MMAs right after the named barrier that completes their operand.
+// Every thread of warps 0-7 and 9 meets each of these barriers once per chunk,
+// also after a wait has given up, so their generations never mix; warp 9
+// reaches them first, so the state warps do not wait there. MMA3 runs while
+// the state warps update S; its completion and the state warps' arrivals
+// release the record stage. D1 is double-buffered in TMEM. The output of chunk
+// c is read out of TMEM at the end of chunk c, once MMA3 is done and the
+// tensor pipe is idle (a TMEM load next to a running MMA slows both), and is
+// stored while MMA1 of chunk c+1 runs.
+constexpr int kCarryThreads = 320;
+constexpr int kCarrySync = 288;      // state warps + the MMA warp
+constexpr uint32_t kTmemCols = 512;  // D1[0]: [0,128), D1[1]: [128,256), D2: [256,384)
 
-enum { kErrFull = 1, kErrEmpty, kErrD1, kErrD2 };
+enum { kErrFull = 1, kErrEmpty, kErrD1, kErrD2, kErrO };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads)
 {
@@ -747,14 +761,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CarrySmem::kBar);
-    uint64_t *full = bars + 0;   // [2]
-    uint64_t *empty = bars + 2;  // [2]
-    uint64_t *d1_done = bars + 4;
-    uint64_t *d2_done = bars + 5;
-    uint64_t *pu_go = bars + 6;    // K^^T U issued: the [0;P] U group may follow
-    uint64_t *pu_done = bars + 7;  // [0;P] U completed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 9);
+    uint64_t *full = bars + 0;     // [2] record landed
+    uint64_t *empty = bars + 2;    // [2] 8 state warps + the MMA3 commit
+    uint64_t *d1_done = bars + 4;  // MMA1 completed
+    uint64_t *d2_done = bars + 5;  // MMA2 completed
+    uint64_t *o_ready = bars + 6;  // MMA3 completed: D1[c & 1] holds O^T of chunk c
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 8);
 
     // one CTA per (sequence, head, half), sequences longest first
     const int H = p.H;
@@ -765,19 +778,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&full[0], 1); tc::mbar_init(&full[1], 1);
-        tc::mbar_init(&empty[0], 8); tc::mbar_init(&empty[1], 8);
-        tc::mbar_init(d1_done, 1); tc::mbar_init(d2_done, 1);
-        tc::mbar_init(pu_go, 1); tc::mbar_init(pu_done, 1);
+        tc::mbar_init(&empty[0], 9); tc::mbar_init(&empty[1], 9);
+        tc::mbar_init(d1_done, 1); tc::mbar_init(d2_done, 1); tc::mbar_init(o_ready, 1);
         *abort = 0;
         tc::fence_mbar_init();
     }
-    // rows 0..63 of the [0; P] operand stay zero
-    for (int s2 = 0; s2 < 2; ++s2) {
-        uint4 *z = reinterpret_cast<uint4 *>(sm + s2 * CarrySmem::kStage + CarrySmem::kA2b);
-        for (int i = threadIdx.x; i < 8192 / 16; i += kCarryThreads) z[i] = make_uint4(0, 0, 0, 0);
-    }
     if (warp == 0) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
-    tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
     tc::tc_fence_after_sync();
@@ -794,166 +800,185 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
                 if (lc >= 2) tc::mbar_wait(&empty[st], ((lc >> 1) - 1) & 1, abort, p.err, kErrEmpty);
                 const uint8_t *rec = p.rec + ((size_t)(c0 + lc) * H + h) * Record::kBytes;
                 uint8_t *sb = sm + st * CarrySmem::kStage;
-                tc::mbar_arrive_expect_tx(&full[st], 32768 + 16384 + 8192 + 512 + 16384);
+                tc::mbar_arrive_expect_tx(&full[st], 32768 + 16384 + 8192 + 16384 + 512);
                 tc::bulk_g2s(sb + CarrySmem::kA1, rec + Record::kA1, 32768, &full[st]);
                 tc::bulk_g2s(sb + CarrySmem::kKh, rec + Record::kKh, 16384, &full[st]);
-                tc::bulk_g2s(sb + CarrySmem::kA2b + 8192, rec + Record::kP, 8192, &full[st]);
-                tc::bulk_g2s(sb + CarrySmem::kG, rec + Record::kG, 512, &full[st]);
+                tc::bulk_g2s(sb + CarrySmem::kP, rec + Record::kP, 8192, &full[st]);
                 tc::bulk_g2s(sb + CarrySmem::kU, rec + Record::kU + half * 16384, 16384, &full[st]);
+                tc::bulk_g2s(sb + CarrySmem::kG, rec + Record::kG, 512, &full[st]);
             }
             // every issued copy has landed before the CTA may exit
             for (int lc = (nc > 2 ? nc - 2 : 0); lc < nc; ++lc)
                 tc::mbar_wait(&full[lc & 1], (lc >> 1) & 1, abort, p.err, kErrFull);
-        } else if (lane == 1) {
-            // The output-only product [0; P] U: queued right behind K^^T U, so the
-            // state update (which waits only for K^^T U) does not wait for it.
-            const uint32_t id2b = tc::idesc_bf16(128, 64, 0, 1);
-            const uint32_t b2 = tc::smem_u32(sm + CarrySmem::kB2);
-            for (int lc = 0; lc < nc; ++lc) {
-                const int st = lc & 1;
-                tc::mbar_wait(pu_go, lc & 1, abort, p.err, kErrD2);
+        }
+    } else if (warp == 9) {
+        // ---------------- MMA issue
+        const uint32_t id1 = tc::idesc_bf16(64, 128, 0, 0);  // S^T . [W; Q~]^T
+        const uint32_t id2 = tc::idesc_bf16(64, 128, 0, 1);  // U^T . K^ (MN-major)
+        const uint32_t id3 = tc::idesc_bf16(64, 64, 0, 0);   // U^T . P^T
+        const uint32_t a_s = tc::smem_u32(sm + CarrySmem::kSt);
+        const uint32_t a_u = tc::smem_u32(sm + CarrySmem::kUt);
+        for (int lc = 0; lc < nc; ++lc) {
+            const int st = lc & 1;
+            const uint32_t sb = tc::smem_u32(sm + st * CarrySmem::kStage);
+            const uint32_t d1 = tmem + (uint32_t)st * 128;
+            if (lane == 0) tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
+            __syncwarp();
+            named_bar(1, kCarrySync);  // S^T complete
+            if (lane == 0) {
                 tc::tc_fence_after_sync();
-                const uint32_t a2b = tc::smem_u32(sm + st * CarrySmem::kStage + CarrySmem::kA2b);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(d1, tc::smem_desc(a_s + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                 tc::smem_desc(sb + CarrySmem::kA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                 id1, kk > 0);
+                tc::mma_commit(d1_done);
+            }
+            __syncwarp();
+            named_bar(2, kCarrySync);  // U^T complete
+            if (lane == 0) {
+                tc::tc_fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + (uint32_t)st * 128, tc::smem_desc(a2b + kk * 32, 16, 1024),
-                                 tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2b, 1);
-                tc::mma_commit(pu_done);
+                    tc::mma_bf16(tmem + 256, tc::smem_desc(a_u + kk * 32, 16, 1024),
+                                 tc::smem_desc(sb + CarrySmem::kKh + kk * 2048, 8192, 1024), id2, kk > 0);
+                tc::mma_commit(d2_done);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(d1 + 64, tc::smem_desc(a_u + kk * 32, 16, 1024),
+                                 tc::smem_desc(sb + CarrySmem::kP + kk * 32, 16, 1024), id3, 1);
+                tc::mma_commit(o_ready);
+                tc::mma_commit(&empty[st]);
             }
+            __syncwarp();
         }
     } else {
         // ---------------- state owners
-        const int lg = warp & 3;                  // TMEM lane group
-        const int t = lg * 32 + lane;             // state row (dk index) / accumulator row
-        const int cb = (warp >> 2) * 32;          // first value column of this thread
-        const uint32_t lane_addr = tmem + ((uint32_t)(lg * 32) << 16);
-        const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 1);   // [W;Q~] K-major . S MN-major
-        const uint32_t id2a = tc::idesc_bf16(128, 64, 1, 1);  // K^^T MN-major . U MN-major
-        const uint32_t b1 = tc::smem_u32(sm + CarrySmem::kB1);
-        const uint32_t b2 = tc::smem_u32(sm + CarrySmem::kB2);
+        const int lg = warp & 3, wh = warp >> 2, hl = lane >> 4;
+        const int cr = 16 * lg + (lane & 15);  // S^T row: value column inside the slice
+        const int kc0 = 64 * wh + 32 * hl;     // first key channel of this thread
+        const int tk0 = 32 * wh + 16 * hl;     // first token of this thread in U^T and O^T
+        const uint32_t lane_base = tmem + ((uint32_t)(lg * 32) << 16);
         float S[32];
-        const size_t sbase = (((size_t)n * H + h) * D + t) * D + half * kSlice + cb;
+        const size_t sbase = ((size_t)n * H + h) * D * D + (size_t)kc0 * D + half * kSlice + cr;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p.S0) x = *reinterpret_cast<const float4 *>(p.S0 + sbase + j);
-            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-        }
-        // bf16 copy of this thread's 32 values into row `row` of a 64-column
-        // MN-major operand (4 of the row's 8 swizzled 16-byte chunks)
-        auto store_bf16 = [&](uint8_t *base, int row, const float *vals) {
+        for (int j = 0; j < 32; ++j) S[j] = p.S0 ? p.S0[sbase + (size_t)j * D] : 0.f;
+        // bf16 S^T row cr, channels kc0..kc0+31: 4 of the row's 8 swizzled
+        // 16-byte chunks in K-block wh
+        auto store_st = [&]() {
+            uint8_t *base = sm + CarrySmem::kSt + wh * 8192;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int q = 0; q < 4; ++q) {
                 uint32_t w[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat162 b = __floats2bfloat162_rn(vals[c4 * 8 + 2 * e],
-                                                             vals[c4 * 8 + 2 * e + 1]);
-                    w[e] = *reinterpret_cast<uint32_t *>(&b);
-                }
-                *reinterpret_cast<uint4 *>(base + tc::sw128(row, (cb / 8 + c4) * 16)) =
+                for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(S[8 * q + 2 * e], S[8 * q + 2 * e + 1]);
+                *reinterpret_cast<uint4 *>(base + tc::sw128(cr, (4 * hl + q) * 16)) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
-        // output rows of chunk lc (lanes 64..127): D1[lc & 1] -> o
-        auto write_o = [&](int lc) {
-            const int r = t - 64;
-            const int t0 = ts + lc * C;
-            float ov[32];
-            tc::tmem_ld32_sync(lane_addr + (lc & 1) * 128 + cb, ov);
-            if (r < min(C, te - t0)) {
-                __nv_bfloat16 *orow = p.o + ((size_t)(t0 + r) * H + h) * D + half * kSlice + cb;
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(p.scale * ov[j + 2 * e],
-                                                                 p.scale * ov[j + 2 * e + 1]);
-                        w[e] = *reinterpret_cast<uint32_t *>(&b);
-                    }
-                    *reinterpret_cast<uint4 *>(orow + j) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
+        // Output of chunk lc: O^T rows in D1[lc & 1], columns 64..127, read into
+        // ov by read_o. store_o sends the warp's 16 value columns x 32 tokens
+        // through a 1 KB staging tile (token rows of 32 bytes, value pairs packed
+        // with one shuffle), then to o with two 16-byte stores per lane: 2 global
+        // store instructions per warp instead of 16, which would slow the
+        // concurrent MMA1.
+        uint8_t *os = sm + CarrySmem::kOs + warp * 1024;
+        float ov[16];
+        auto read_o = [&](int lc) {
+            tc::mbar_wait(o_ready, lc & 1, abort, p.err, kErrO);
+            tc::tc_fence_after_sync();
+            tc::tmem_ld16x2_x16_sync(lane_base + (uint32_t)(lc & 1) * 128 + 64 + 32 * wh, ov);
         };
-        store_bf16(sm + CarrySmem::kB1, t, S);
+        auto store_o = [&](int lc) {
+            const bool odd = lane & 1;
+            const int l15 = lane & 15;
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                // even lane: token j, columns (l15, l15+1); odd lane: token j+1, (l15-1, l15)
+                const float x = __shfl_xor_sync(0xffffffffu, odd ? ov[j] : ov[j + 1], 1);
+                const int row = 16 * hl + j + (odd ? 1 : 0);
+                const uint32_t w = odd ? pack_bf16x2(p.scale * x, p.scale * ov[j + 1])
+                                       : pack_bf16x2(p.scale * ov[j], p.scale * x);
+                *reinterpret_cast<uint32_t *>(os + row * 32 + (l15 & ~1) * 2) = w;
+            }
+            __syncwarp();
+            const int t0 = ts + lc * C;
+            const int L = min(C, te - t0);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int k = lane + 32 * i;           // 16-byte piece: token row k/2, half k&1
+                const int tok = 32 * wh + (k >> 1);
+                if (tok < L)
+                    *reinterpret_cast<uint4 *>(p.o + ((size_t)(t0 + tok) * H + h) * D + half * kSlice +
+                                               16 * lg + 8 * (k & 1)) =
+                        *reinterpret_cast<const uint4 *>(os + k * 16);
+            }
+            __syncwarp();
+        };
+        store_st();
         tc::fence_proxy_async_smem();
-        tc::tc_fence_before_sync();
 
         for (int lc = 0; lc < nc; ++lc) {
             const int st = lc & 1;
-            uint8_t *sb = sm + st * CarrySmem::kStage;
-            const uint32_t d1 = tmem + (uint32_t)st * 128;  // this chunk's output accumulator
-            // A. the bf16 state is complete: issue MMA1 = [W; Q~] . S
-            named_bar(1, 256);
-            if (threadIdx.x == 0) {
-                tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
-                tc::tc_fence_after_sync();
-                const uint32_t sbase_a = tc::smem_u32(sb + CarrySmem::kA1);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(d1, tc::smem_desc(sbase_a + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                 tc::smem_desc(b1 + kk * 2048, 8192, 1024), id1, kk > 0);
-                tc::mma_commit(d1_done);
-            }
-            // E. previous chunk's output rows, off the critical path
-            if (lg >= 2 && lc > 0) write_o(lc - 1);
+            const uint8_t *sb = sm + st * CarrySmem::kStage;
+            // A. S^T is complete: MMA1 may go
+            tc::tc_fence_before_sync();
+            named_bar(1, kCarrySync);
+            // B. previous chunk's output, while MMA1 runs
+            if (lc > 0) store_o(lc - 1);
+            // C. U^T = U~^T - (W S)^T for tokens tk0..tk0+15
             tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
-            if (lg < 2) {
-                // C. U = U~ - W S for tokens 0..63, then MMA2
-                tc::mbar_wait(d1_done, lc & 1, abort, p.err, kErrD1);
-                tc::tc_fence_after_sync();
-                float U[32];
-                tc::tmem_ld32_sync(lane_addr + (uint32_t)st * 128 + cb, U);
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 ut = *reinterpret_cast<const float4 *>(
-                        sb + CarrySmem::kU + u_swz(t, cb + j));
-                    U[j] = ut.x - U[j]; U[j + 1] = ut.y - U[j + 1];
-                    U[j + 2] = ut.z - U[j + 2]; U[j + 3] = ut.w - U[j + 3];
-                }
-                store_bf16(sm + CarrySmem::kB2, t, U);
-                tc::fence_proxy_async_smem();
-                tc::tc_fence_before_sync();
-                named_bar(2, 128);
-                if (threadIdx.x == 0) {
-                    tc::tc_fence_after_sync();
-                    const uint32_t kh = tc::smem_u32(sb + CarrySmem::kKh);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(tmem + 64, tc::smem_desc(kh + kk * 2048, 8192, 1024),
-                                     tc::smem_desc(b2 + kk * 2048, 8192, 1024), id2a, kk > 0);
-                    tc::mma_commit(d2_done);
-                    tc::mbar_arrive(pu_go);
-                }
-            }
-            // D. S = gamma * S + K^^T U, and its bf16 copy for the next MMA1
-            tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2);
+            tc::mbar_wait(d1_done, lc & 1, abort, p.err, kErrD1);
             tc::tc_fence_after_sync();
             {
-                float ku[32];
-                tc::tmem_ld32_sync(tmem + 64 + ((uint32_t)(lg * 32) << 16) + cb, ku);
-                const float gamma = reinterpret_cast<const float *>(sb + CarrySmem::kG)[t];
+                float U[16];
+                tc::tmem_ld16x2_x16_sync(lane_base + (uint32_t)st * 128 + 32 * wh, U);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = gamma * S[j] + ku[j];
+                for (int m = 0; m < 4; ++m) {
+                    const float4 ut = *reinterpret_cast<const float4 *>(
+                        sb + CarrySmem::kU + u_swz(cr, tk0 + 4 * m));
+                    U[4 * m] = ut.x - U[4 * m]; U[4 * m + 1] = ut.y - U[4 * m + 1];
+                    U[4 * m + 2] = ut.z - U[4 * m + 2]; U[4 * m + 3] = ut.w - U[4 * m + 3];
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(U[8 * q + 2 * e], U[8 * q + 2 * e + 1]);
+                    *reinterpret_cast<uint4 *>(sm + CarrySmem::kUt + tc::sw128(cr, (tk0 / 8 + q) * 16)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
             }
-            store_bf16(sm + CarrySmem::kB1, t, S);
             tc::fence_proxy_async_smem();
             tc::tc_fence_before_sync();
-            // [0;P] U (another thread's commit) has finished reading this stage and
-            // B2 and adding into D1[st]: the stage can go back to the producer, the
-            // next chunk may rewrite B2 and write_o may read D1[st]
-            tc::mbar_wait(pu_done, lc & 1, abort, p.err, kErrD2);
-            tc::tc_fence_after_sync();
+            named_bar(2, kCarrySync);
+            // D. S^T = S^T Diag(gamma) + D2, and its bf16 copy for the next MMA1
+            {
+                float g[32];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sb + CarrySmem::kG + (kc0 + j) * 4);
+                    g[j] = x.x; g[j + 1] = x.y; g[j + 2] = x.z; g[j + 3] = x.w;
+                }
+                tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2);
+                tc::tc_fence_after_sync();
+                float ku[32];
+                tc::tmem_ld16x2_x32_sync(lane_base + 256 + 64 * wh, ku);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = g[j] * S[j] + ku[j];
+            }
+            store_st();
+            tc::fence_proxy_async_smem();
+            // this warp has read its last piece of the stage (U~^T, gamma)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&empty[st]);
+            // E. this chunk's output, once MMA3 is done
+            read_o(lc);
         }
-        if (lg >= 2 && nc > 0) write_o(nc - 1);
+        if (nc > 0) store_o(nc - 1);
         if (p.S_final) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4 *>(p.S_final + sbase + j) =
-                    make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            for (int j = 0; j < 32; ++j) p.S_final[sbase + (size_t)j * D] = S[j];
         }
     }
     tc::tc_fence_before_sync();
