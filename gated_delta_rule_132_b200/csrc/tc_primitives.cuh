@@ -86,13 +86,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
                  : "memory");
 }
 
-// Hint to bring `bytes` of global memory into L2 (no destination, no
-// completion to wait for). Address 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src_gmem, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes) : "memory");
-}
-
 // 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of
 // this thread's outstanding copies.
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem)
