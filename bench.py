@@ -44,7 +44,7 @@ LAUNCHES_PER_PREFILL = 4
 # traffic grows in proportion to the records a launch processes. Sources:
 # profiles/tc_prep2_kernel_chunked_B4_H16_T4096.md and
 # profiles/tc_carry_kernel_chunked_B4_H16_T4096.md.
-TRAFFIC_PER_RECORD = {"prepare": 162_774, "carry": 105_200}
+TRAFFIC_PER_RECORD = {"prepare": 162_304, "carry": 105_469}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
