@@ -239,6 +239,44 @@ def bench_decode(P, steps, warmup, world, rank, dev):
     return dict(ms=ms, kern_ms=kern_ms, bytes=state_b + io_b, state_bytes=state_b)
 
 
+DECODE_TOKENS_T = 8  # tokens per multi-token decode call
+
+
+def bench_decode_tokens(P, T, steps, warmup, world, rank, dev):
+    """kda_decode_tokens on the decode workload's state with T tokens per call;
+    four input sets of the call's shape are cycled (the 537 MB state, touched
+    once each way per call, dominates the bytes)."""
+    from gated_delta_rule_132_b200 import kda
+    devs = f"cuda:{dev}"
+    S = I.make_decode_state(P.N, P.H, P.d, P.s_std, P.seed + 2000 + 1000 * rank, device=devs)
+    names = ("q", "k", "v", "log_alpha", "beta")
+    pool = []
+    for i in range(4):
+        x = I.make_prefill(P.N, T, P.H, P.d, P.dtype, gate_shift=P.gate_shift,
+                           seed=P.step_seed0 + 50000 + i + 100000 * rank, device=devs)
+        pool.append({n: x[n] for n in names})
+    o = torch.empty(P.N, T, P.H, P.d, dtype=P.dtype, device=devs)
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        kda.kda_decode_tokens(**pool[i % 4], S=S, o=o)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    def step(i, ev):
+        ev[0].record(stream)
+        kda.kda_decode_tokens(**pool[i % 4], S=S, o=o)
+        ev[1].record(stream)
+
+    total_ms, per = time_region(step, steps, stream, marks=2)
+    barrier(world)
+    ms = max_over_ranks(total_ms / steps, world)
+    kern_ms = statistics.mean(p[0] for p in per)
+    units = P.N * P.H
+    state_b = 2 * units * P.d * P.d * 4
+    io_b = units * T * (3 * P.d * 2 + 4 * P.d + 4 + P.d * 2)
+    return dict(ms=ms, kern_ms=kern_ms, bytes=state_b + io_b, T=T, tokens=P.N * T)
+
+
 def bench_e2e(pre, steps, stream):
     """The same prefill through the public call with host buffers: pinned host
     inputs copied in, kda_chunk_fwd, o and S_final copied out, every step."""
@@ -303,6 +341,8 @@ def run_ours(args, world, rank, dev):
         pre = bench_prefill(preset, args.steps, args.warmup, world, rank, dev, peaks)
         dec = None if args.no_decode else bench_decode(I.DECODE, args.steps, args.warmup,
                                                        world, rank, dev)
+        dtok = None if args.no_decode else bench_decode_tokens(
+            I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
     hbm = peaks["hbm_gbs"]
     value = pre["tokens"] * world / (pre["ms"] / 1e3)
 
@@ -354,6 +394,18 @@ def run_ours(args, world, rank, dev):
                                        "achieved": round(dec_ach, 1), "peak": hbm,
                                        "unit": "GB/s", "frac": round(dec_ach / hbm, 4),
                                        "traffic": None, "bytes_per_launch": dec["bytes"]}}
+    if dtok is not None:
+        t_ach = dtok["bytes"] / (dtok["kern_ms"] / 1e3) / 1e9
+        line["decode_tokens"] = {
+            "workload": f"{I.DECODE.name}_T{dtok['T']}", "value": round(t_ach, 1),
+            "unit": "GB/s", "tokens_per_s": round(dtok["tokens"] / (dtok["kern_ms"] / 1e3), 1),
+            "ms_per_call": round(dtok["kern_ms"], 4),
+            "vs_single_steps": (round(dtok["T"] * dec["kern_ms"] / dtok["kern_ms"], 3)
+                                if dec is not None else None),
+            "roofline": {"kernel": "decode (T tokens per call)", "bound": "hbm",
+                         "achieved": round(t_ach, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(t_ach / hbm, 4), "traffic": None,
+                         "bytes_per_launch": dtok["bytes"]}}
     c = clocks.summary()
     line["clocks"] = c
     if not args.no_e2e:

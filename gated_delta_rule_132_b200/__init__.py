@@ -1,7 +1,8 @@
 """Kimi Delta Attention (KDA) on NVIDIA B200: a C-ABI CUDA library (sm_100a)
 with a thin Python binding.
 
-The compute entry points (``kda_chunk_fwd``, ``kda_decode_step``) live in
+The compute entry points (``kda_chunk_fwd``, ``kda_decode_step``,
+``kda_decode_tokens``) live in
 ``gated_delta_rule_132_b200.kda`` and load the in-tree ``libkda_b200.so`` on
 first use; ``inputs`` holds the seeded synthetic-input generators.
 """
@@ -10,8 +11,8 @@ import importlib
 from . import inputs  # noqa: F401  (no CUDA needed)
 
 _EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_prepare", "kda_chunk_fwd_carry",
-            "kda_decode_step", "kda_chunk_fwd_workspace_size", "ChunkFwdCall", "lib",
-            "KdaError")
+            "kda_decode_step", "kda_decode_tokens", "kda_chunk_fwd_workspace_size",
+            "ChunkFwdCall", "lib", "KdaError")
 
 
 def __getattr__(name):

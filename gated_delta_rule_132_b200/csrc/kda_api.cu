@@ -161,21 +161,33 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtyp
                             KDA_ALGO_AUTO, stream);
 }
 
+kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                               const float *log_alpha, const float *beta, float *S, int N,
+                               int T, int H, int dk, int dv, float scale, void *o,
+                               void *stream)
+{
+    if (N < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || !head_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * T > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if (!S) return KDA_ERR_INVALID_ARG;
+    if (T == 0) return KDA_OK;  // no token: S unchanged, nothing launched
+    if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
+    const cudaError_t e = kda::launch_decode(q, k, v, dt, log_alpha, beta, S, N, T, H, dk, dv,
+                                             scale, o, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t dt,
                              const float *log_alpha, const float *beta, float *S, int N,
                              int H, int dk, int dv, float scale, void *o, void *stream)
 {
-    if (N < 1 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
-    if (!dtype_ok(dt) || !head_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
-    if ((long long)N * H > (long long)INT32_MAX) return KDA_ERR_UNSUPPORTED;
-    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
-    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
-    for (const void *ptr : ptrs)
-        if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
-    const cudaError_t e = kda::launch_decode(q, k, v, dt, log_alpha, beta, S, N, H, dk, dv,
-                                             scale, o, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda_decode_tokens(q, k, v, dt, log_alpha, beta, S, N, 1, H, dk, dv, scale, o,
+                             stream);
 }
 
 }  // extern "C"

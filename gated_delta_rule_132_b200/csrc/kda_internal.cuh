@@ -64,9 +64,11 @@ WorkspaceLayout simt_workspace_layout(const Problem &p);
 WorkspaceLayout tc_workspace_layout(const Problem &p);
 
 cudaError_t launch_plan(const Problem &p, Plan plan, cudaStream_t stream);
+// T tokens per (sequence, head): q, k, log_alpha [N, T, H, dk], v, o [N, T, H, dv],
+// beta [N, T, H]; S [N, H, dk, dv] read once and written once.
 cudaError_t launch_decode(const void *q, const void *k, const void *v, kda_dtype_t dt,
-                          const float *log_alpha, const float *beta, float *S, int N, int H,
-                          int dk, int dv, float scale, void *o, cudaStream_t stream);
+                          const float *log_alpha, const float *beta, float *S, int N, int T,
+                          int H, int dk, int dv, float scale, void *o, cudaStream_t stream);
 // Prefill phases: bit 0 = prepare (plan + chunk-parallel kernel), bit 1 = carry.
 enum : int { kPhasePrepare = 1, kPhaseCarry = 2, kPhaseAll = 3 };
 cudaError_t launch_simt_prefill(const Problem &p, void *workspace, int phases,

@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.kda_decode_step.restype = _i
         L.kda_decode_step.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                                       _vp, _vp]
+        L.kda_decode_tokens.restype = _i
+        L.kda_decode_tokens.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                        _f, _vp, _vp]
         _lib = L
     return _lib
 
@@ -220,4 +223,33 @@ def kda_decode_step(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None
                                N, H, dk, dv, float(scale), _p(o), _stream(stream))
     if st != 0:
         raise KdaError("kda_decode_step", st)
+    return o
+
+
+def kda_decode_tokens(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None):
+    """T recurrent decode steps in one call (C: ``kda_decode_tokens``); updates S in place.
+
+    q, k [N,T,H,dk]; v [N,T,H,dv] (bf16 or fp32); log_alpha [N,T,H,dk] fp32;
+    beta [N,T,H] fp32; S [N,H,dk,dv] fp32. Returns o [N,T,H,dv] in q's dtype.
+    """
+    N, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dtype = q.dtype
+    _dt(q)
+    _need(q, "q", dtype, (N, T, H, dk))
+    _need(k, "k", dtype, (N, T, H, dk))
+    _need(v, "v", dtype, (N, T, H, dv))
+    _need(log_alpha, "log_alpha", torch.float32, (N, T, H, dk))
+    _need(beta, "beta", torch.float32, (N, T, H))
+    _need(S, "S", torch.float32, (N, H, dk, dv))
+    if scale is None:
+        scale = dk ** -0.5
+    if o is None:
+        o = torch.empty((N, T, H, dv), dtype=dtype, device=q.device)
+    else:
+        _need(o, "o", dtype, (N, T, H, dv))
+    st = lib().kda_decode_tokens(_p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S),
+                                 N, T, H, dk, dv, float(scale), _p(o), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_decode_tokens", st)
     return o

@@ -168,6 +168,26 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dt
                              int H, int dk, int dv, float scale, void *o, void *stream);
 
 /*
+ * Multi-token decode: T new tokens for each of N independent sequences, applied
+ * in order with the state held on chip between them; S is read once and
+ * written once per call. Source: the same update rule, applied T times (each
+ * token as in kda_decode_step). Equals T chained kda_decode_step calls, and
+ * kda_chunk_fwd with B = N, S0 = S_final = S (up to rounding); meant for small
+ * T (speculative verification, continuing a prefill by a few tokens), where the
+ * chunked prefill would spend most of its time on per-chunk intermediates.
+ *
+ *   q, k        qkv_dtype [N, T, H, dk]   v, o   qkv_dtype [N, T, H, dv]
+ *   log_alpha   fp32 [N, T, H, dk]        beta   fp32 [N, T, H]
+ *   S           fp32 [N, H, dk, dv], read and overwritten
+ * Errors as kda_decode_step; T = 0 returns KDA_OK without touching anything
+ * (only S must then be non-null). N * T must fit in a signed 32-bit int.
+ */
+kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v,
+                               kda_dtype_t qkv_dtype, const float *log_alpha,
+                               const float *beta, float *S, int N, int T, int H, int dk,
+                               int dv, float scale, void *o, void *stream);
+
+/*
  * kda_chunk_fwd_noalloc — the chunked prefill for callers that cannot allocate
  * device memory (no counterpart in the paper; it exists for callers such as a
  * plugin whose host application owns all device memory, or code that must not

@@ -27,8 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for required in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
-                     "kda_status_string"):
+    for required in ("kda_chunk_fwd", "kda_decode_step", "kda_decode_tokens",
+                     "kda_chunk_fwd_workspace_size", "kda_status_string"):
         assert required in names
 
 
@@ -94,6 +94,22 @@ def test_decode_rejects(L, kw, status):
     assert L.kda_decode_step(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["S"],
                              a["N"], a["H"], a["dk"], a["dv"], a["scale"], a["o"],
                              a["stream"]) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=0), 1), (dict(T=-1), 1), (dict(S=None), 1), (dict(q=None), 1), (dict(o=None), 1),
+    (dict(dk=48, dv=48), 2), (dict(dt=3), 2), (dict(N=1 << 20, T=1 << 12), 2),
+    (dict(S=_fake(0x10008)), 3), (dict(v=_fake(0x10002)), 3), (dict(scale=float("nan")), 1),
+    # no token: nothing is read, written or launched, and only S must be given
+    (dict(T=0, q=None, k=None, v=None, la=None, beta=None, o=None), 0),
+])
+def test_decode_tokens_rejects(L, kw, status):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), dt=1, la=_fake(), beta=_fake(), S=_fake(),
+             N=4, T=3, H=2, dk=128, dv=128, scale=0.1, o=_fake(), stream=None)
+    a.update(kw)
+    assert L.kda_decode_tokens(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["S"],
+                               a["N"], a["T"], a["H"], a["dk"], a["dv"], a["scale"], a["o"],
+                               a["stream"]) == status
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -65,3 +65,86 @@ def test_decode_is_deterministic():
     o1 = kda.kda_decode_step(**tok, S=S1)
     o2 = kda.kda_decode_step(**tok, S=S2)
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+# ----------------------------------------------------------------- multi-token decode
+def _tokens_problem(N, T, H, d, dtype, seed):
+    x = I.make_prefill(N, T, H, d, dtype, gate_shift=-2.0, seed=seed)
+    S = I.make_decode_state(N, H, d, 0.05, seed=seed + 1)
+    return x, S
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T", [1, 2, 7, 33])
+def test_decode_tokens_vs_oracle(T, dtype, d):
+    """T tokens in one call against the fp64 token-by-token forward started from S."""
+    N, H = 3, 2
+    x, S = _tokens_problem(N, T, H, d, dtype, seed=300 + T + d)
+    S_gpu = S.cuda()
+    o = kda.kda_decode_tokens(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(),
+                              x["log_alpha"].cuda(), x["beta"].cuda(), S_gpu, scale=x["scale"])
+    o_ref, S_ref = oracle.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S0=S,
+                                  scale=x["scale"])
+    assert o.shape == (N, T, H, d)
+    assert rel_l2(o, o_ref) <= TOL[dtype]
+    assert rel_l2(S_gpu, S_ref) <= TOL[torch.float32]
+
+
+def test_decode_tokens_equals_chained_steps():
+    """One T-token call and T single-step calls run the same per-token arithmetic
+    on the same fp32 state, so they agree bit for bit."""
+    N, T, H, d = 4, 5, 3, 128
+    x, S = _tokens_problem(N, T, H, d, torch.bfloat16, seed=41)
+    g = {k: v.cuda() for k, v in x.items() if isinstance(v, torch.Tensor)}
+    S1, S2 = S.cuda(), S.cuda()
+    o1 = kda.kda_decode_tokens(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S1,
+                               scale=x["scale"])
+    for t in range(T):
+        o2 = kda.kda_decode_step(g["q"][:, t].contiguous(), g["k"][:, t].contiguous(),
+                                 g["v"][:, t].contiguous(), g["log_alpha"][:, t].contiguous(),
+                                 g["beta"][:, t].contiguous(), S2, scale=x["scale"])
+        assert torch.equal(o1[:, t], o2), t
+    assert torch.equal(S1, S2)
+
+
+def test_decode_tokens_matches_prefill_continuation():
+    """Continuing from a state with T tokens equals the chunked prefill with
+    S0 = that state (both within the bf16 tolerance of the oracle)."""
+    N, T, H, d = 2, 24, 4, 128
+    x, S = _tokens_problem(N, T, H, d, torch.bfloat16, seed=52)
+    g = {k: v.cuda() for k, v in x.items() if isinstance(v, torch.Tensor)}
+    S_dec = S.cuda()
+    o_dec = kda.kda_decode_tokens(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S_dec,
+                                  scale=x["scale"])
+    o_pre, S_pre = kda.kda_chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"],
+                                     S0=S.cuda(), scale=x["scale"])
+    assert rel_l2(o_dec, o_pre.float().cpu()) <= TOL[torch.bfloat16]
+    assert rel_l2(S_dec, S_pre.cpu()) <= 1e-2
+
+
+def test_decode_tokens_zero_tokens_leaves_state():
+    N, H, d = 2, 2, 64
+    S = I.make_decode_state(N, H, d, 0.05, seed=9).cuda()
+    S0 = S.clone()
+    e = torch.empty((N, 0, H, d), device="cuda")
+    o = kda.kda_decode_tokens(e, e, e, e, torch.empty((N, 0, H), device="cuda"), S)
+    assert o.shape == (N, 0, H, d) and torch.equal(S, S0)
+
+
+def test_decode_tokens_full_batch_sampled():
+    """Decode workload shape (256 sequences x 32 heads, d=128) with 8 tokens per
+    call; a seeded subset of 16 sequences is checked against the oracle (units
+    are independent, so the subset is exact)."""
+    P = I.DECODE
+    T = 8
+    x = I.make_prefill(P.N, T, P.H, P.d, P.dtype, gate_shift=P.gate_shift, seed=77)
+    S = I.make_decode_state(P.N, P.H, P.d, P.s_std, P.seed)
+    subset = torch.randperm(P.N, generator=torch.Generator().manual_seed(8))[:16].sort().values
+    S_gpu = S.cuda()
+    o = kda.kda_decode_tokens(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(),
+                              x["log_alpha"].cuda(), x["beta"].cuda(), S_gpu, scale=x["scale"])
+    sub = {k: x[k][subset] for k in ("q", "k", "v", "log_alpha", "beta")}
+    o_ref, S_ref = oracle.forward(**sub, S0=S[subset], scale=x["scale"])
+    assert rel_l2(o[subset.cuda()], o_ref) <= TOL[P.dtype]
+    assert rel_l2(S_gpu[subset.cuda()], S_ref) <= 1e-4
