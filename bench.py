@@ -210,6 +210,37 @@ def bench_prefill(preset, steps, warmup, world, rank, dev, peaks):
                 records=chunks * preset.H)
 
 
+def bench_gdn(pre, steps, warmup, world):
+    """The same prefill with one gate per token and head (kda_gdn_chunk_fwd): the
+    gate is channel 0 of the workload's per-channel gate; the KDA call's
+    workspace is reused."""
+    from gated_delta_rule_132_b200 import kda
+    x = pre["x"]
+    la = x["log_alpha"][..., 0].contiguous()
+    call = kda.ChunkFwdCall(x["q"], x["k"], x["v"], la, x["beta"], x["S0"], x["cu_seqlens"],
+                            x["scale"], workspace=pre["call"].workspace, gate="head")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        call.run()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    def step(i, ev):
+        ev[0].record(stream)
+        call.prepare()
+        ev[1].record(stream)
+        call.carry()
+        ev[2].record(stream)
+
+    total_ms, per = time_region(step, steps, stream, marks=3)
+    barrier(world)
+    d = x["q"].shape[-1]
+    in_b = pre["token_heads"] * (3 * d * x["q"].element_size() + 4 + 4)
+    return dict(ms=max_over_ranks(total_ms / steps, world),
+                prep_ms=statistics.mean(p[0] for p in per),
+                carry_ms=statistics.mean(p[1] for p in per), in_bytes=in_b)
+
+
 def bench_decode(P, steps, warmup, world, rank, dev):
     from gated_delta_rule_132_b200 import kda
     devs = f"cuda:{dev}"
@@ -343,6 +374,7 @@ def run_ours(args, world, rank, dev):
                                                        world, rank, dev)
         dtok = None if args.no_decode else bench_decode_tokens(
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
+        gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
     hbm = peaks["hbm_gbs"]
     value = pre["tokens"] * world / (pre["ms"] / 1e3)
 
@@ -406,6 +438,17 @@ def run_ours(args, world, rank, dev):
                          "achieved": round(t_ach, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(t_ach / hbm, 4), "traffic": None,
                          "bytes_per_launch": dtok["bytes"]}}
+    if gdn is not None:
+        g_ach = (gdn["in_bytes"] + ws_per_launch) / (gdn["prep_ms"] / 1e3) / 1e9
+        line["gdn"] = {
+            "workload": preset.name + "_gate_per_head",
+            "value": round(pre["tokens"] * world / (gdn["ms"] / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(gdn["ms"], 4),
+            "kernels_ms": {"prepare": round(gdn["prep_ms"], 4), "carry": round(gdn["carry_ms"], 4)},
+            "roofline": {"kernel": "prepare (one gate per head)", "bound": "hbm",
+                         "achieved": round(g_ach, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(g_ach / hbm, 4), "traffic": None,
+                         "bytes_per_launch": gdn["in_bytes"] + ws_per_launch}}
     c = clocks.summary()
     line["clocks"] = c
     if not args.no_e2e:
@@ -471,6 +514,8 @@ def main():
     ap.add_argument("--workload", choices=["long", "chunked", "varlen"], default="long",
                     help="prefill workload (default: the long-context one)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-gdn", action="store_true",
+                    help="skip the one-gate-per-head (GDN) variant of the prefill")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

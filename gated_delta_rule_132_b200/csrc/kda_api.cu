@@ -32,6 +32,7 @@ kda_status_t describe(int B, int T, int H, int dk, int dv, int n_seqs, bool varl
     p->N = N; p->B = B; p->T = T; p->H = H; p->dk = dk; p->dv = dv; p->dtype = dt;
     p->total_tokens = total;
     p->max_chunks = (int)chunks;
+    p->gate_per_channel = 1;
     return KDA_OK;
 }
 
@@ -90,7 +91,7 @@ static kda_status_t chunk_fwd_phases(const void *q, const void *k, const void *v
                                      const int32_t *cu_seqlens, int n_seqs, int B, int T,
                                      int H, int dk, int dv, float scale, void *o,
                                      float *S_final, void *workspace, size_t workspace_bytes,
-                                     int algo, int phases, void *stream)
+                                     int algo, int phases, int gate_per_channel, void *stream)
 {
     if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TCGEN05)
         return KDA_ERR_INVALID_ARG;
@@ -111,6 +112,7 @@ static kda_status_t chunk_fwd_phases(const void *q, const void *k, const void *v
 
     p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.S0 = S0;
     p.cu_seqlens = cu_seqlens; p.scale = scale; p.o = o; p.S_final = S_final;
+    p.gate_per_channel = gate_per_channel;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = tc ? kda::launch_tc_prefill(p, workspace, phases, s)
                              : kda::launch_simt_prefill(p, workspace, phases, s);
@@ -128,7 +130,27 @@ kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, kda_d
                               int dk, int dv, float scale, void *o, float *S_final,
                               void *workspace, size_t workspace_bytes, int algo, void *stream)
 {
-    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseAll, stream);
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseAll, 1, stream);
+}
+
+kda_status_t kda_gdn_chunk_fwd(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                               const float *log_alpha, const float *beta, const float *S0,
+                               const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                               int dk, int dv, float scale, void *o, float *S_final,
+                               void *workspace, size_t workspace_bytes, int algo, void *stream)
+{
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseAll, 0, stream);
+}
+
+kda_status_t kda_gdn_chunk_fwd_prepare(const void *q, const void *k, const void *v,
+                                       kda_dtype_t dt, const float *log_alpha,
+                                       const float *beta, const float *S0,
+                                       const int32_t *cu_seqlens, int n_seqs, int B, int T,
+                                       int H, int dk, int dv, float scale, void *o,
+                                       float *S_final, void *workspace, size_t workspace_bytes,
+                                       int algo, void *stream)
+{
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhasePrepare, 0, stream);
 }
 
 kda_status_t kda_chunk_fwd_prepare(const void *q, const void *k, const void *v, kda_dtype_t dt,
@@ -138,7 +160,7 @@ kda_status_t kda_chunk_fwd_prepare(const void *q, const void *k, const void *v, 
                                    void *workspace, size_t workspace_bytes, int algo,
                                    void *stream)
 {
-    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhasePrepare, stream);
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhasePrepare, 1, stream);
 }
 
 kda_status_t kda_chunk_fwd_carry(const void *q, const void *k, const void *v, kda_dtype_t dt,
@@ -147,7 +169,7 @@ kda_status_t kda_chunk_fwd_carry(const void *q, const void *k, const void *v, kd
                                  int dk, int dv, float scale, void *o, float *S_final,
                                  void *workspace, size_t workspace_bytes, int algo, void *stream)
 {
-    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseCarry, stream);
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseCarry, 1, stream);
 }
 
 kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtype_t dt,
@@ -161,10 +183,12 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtyp
                             KDA_ALGO_AUTO, stream);
 }
 
-kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t dt,
-                               const float *log_alpha, const float *beta, float *S, int N,
-                               int T, int H, int dk, int dv, float scale, void *o,
-                               void *stream)
+}  // extern "C"
+
+static kda_status_t decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                                  const float *log_alpha, const float *beta, float *S, int N,
+                                  int T, int H, int dk, int dv, float scale, void *o,
+                                  int gate_per_channel, void *stream)
 {
     if (N < 1 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
     if (!dtype_ok(dt) || !head_ok(dk, dv)) return KDA_ERR_UNSUPPORTED;
@@ -178,8 +202,27 @@ kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v, kda_
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
     const cudaError_t e = kda::launch_decode(q, k, v, dt, log_alpha, beta, S, N, T, H, dk, dv,
-                                             scale, o, static_cast<cudaStream_t>(stream));
+                                             scale, o, gate_per_channel,
+                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" {
+
+kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                               const float *log_alpha, const float *beta, float *S, int N,
+                               int T, int H, int dk, int dv, float scale, void *o,
+                               void *stream)
+{
+    return decode_tokens(q, k, v, dt, log_alpha, beta, S, N, T, H, dk, dv, scale, o, 1, stream);
+}
+
+kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                                   const float *log_alpha, const float *beta, float *S, int N,
+                                   int T, int H, int dk, int dv, float scale, void *o,
+                                   void *stream)
+{
+    return decode_tokens(q, k, v, dt, log_alpha, beta, S, N, T, H, dk, dv, scale, o, 0, stream);
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t dt,

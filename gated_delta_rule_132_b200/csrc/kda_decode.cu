@@ -31,7 +31,8 @@ template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, int T, int H, float scale, TIn *__restrict__ o)
+              float *__restrict__ S, int T, int H, int gate_per_channel, float scale,
+              TIn *__restrict__ o)
 {
     constexpr int CG = DV / 4;                  // float4 column groups per row
     constexpr int RG = kDecodeThreads / CG;     // row groups
@@ -63,7 +64,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     auto fetch = [&](int t) {
         const size_t tok = ((size_t)n * T + t) * H + h;  // (n, t, h) of [N, T, H, ...]
         if (tid < DK) {
-            nla = log_alpha[tok * DK + tid];
+            nla = gate_per_channel ? log_alpha[tok * DK + tid] : log_alpha[tok];
             nk = to_f32(k[tok * DK + tid]);
             nq = to_f32(q[tok * DK + tid]);
         }
@@ -128,24 +129,24 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 
 template <int D, typename TIn>
 cudaError_t launch_d(const void *q, const void *k, const void *v, const float *la,
-                     const float *beta, float *S, int units, int T, int H, float scale, void *o,
-                     cudaStream_t st)
+                     const float *beta, float *S, int units, int T, int H, int gpc, float scale,
+                     void *o, cudaStream_t st)
 {
     decode_kernel<D, D, TIn><<<units, kDecodeThreads, 0, st>>>(
         static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v),
-        la, beta, S, T, H, scale, static_cast<TIn *>(o));
+        la, beta, S, T, H, gpc, scale, static_cast<TIn *>(o));
     return cudaGetLastError();
 }
 
 template <typename TIn>
 cudaError_t launch_t(int d, const void *q, const void *k, const void *v, const float *la,
-                     const float *beta, float *S, int units, int T, int H, float scale, void *o,
-                     cudaStream_t st)
+                     const float *beta, float *S, int units, int T, int H, int gpc, float scale,
+                     void *o, cudaStream_t st)
 {
     switch (d) {
-    case 32: return launch_d<32, TIn>(q, k, v, la, beta, S, units, T, H, scale, o, st);
-    case 64: return launch_d<64, TIn>(q, k, v, la, beta, S, units, T, H, scale, o, st);
-    case 128: return launch_d<128, TIn>(q, k, v, la, beta, S, units, T, H, scale, o, st);
+    case 32: return launch_d<32, TIn>(q, k, v, la, beta, S, units, T, H, gpc, scale, o, st);
+    case 64: return launch_d<64, TIn>(q, k, v, la, beta, S, units, T, H, gpc, scale, o, st);
+    case 128: return launch_d<128, TIn>(q, k, v, la, beta, S, units, T, H, gpc, scale, o, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -154,14 +155,16 @@ cudaError_t launch_t(int d, const void *q, const void *k, const void *v, const f
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, kda_dtype_t dt,
                           const float *log_alpha, const float *beta, float *S, int N, int T,
-                          int H, int dk, int dv, float scale, void *o, cudaStream_t stream)
+                          int H, int dk, int dv, float scale, void *o, int gate_per_channel,
+                          cudaStream_t stream)
 {
     if (dk != dv) return cudaErrorInvalidValue;
     const int units = N * H;
     if (dt == KDA_DTYPE_BF16)
-        return launch_t<__nv_bfloat16>(dk, q, k, v, log_alpha, beta, S, units, T, H, scale, o,
-                                       stream);
-    return launch_t<float>(dk, q, k, v, log_alpha, beta, S, units, T, H, scale, o, stream);
+        return launch_t<__nv_bfloat16>(dk, q, k, v, log_alpha, beta, S, units, T, H,
+                                       gate_per_channel, scale, o, stream);
+    return launch_t<float>(dk, q, k, v, log_alpha, beta, S, units, T, H, gate_per_channel,
+                           scale, o, stream);
 }
 
 }  // namespace kda

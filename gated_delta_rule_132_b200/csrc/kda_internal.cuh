@@ -37,6 +37,7 @@ struct Problem {
     kda_dtype_t dtype;
     long long total_tokens;     // B * T (packed time axis length)
     int max_chunks;             // upper bound on chunks over all sequences
+    int gate_per_channel;       // 1: log_alpha [.., H, dk] (KDA); 0: [.., H] (one gate per head)
 };
 
 // Sequence plan in the workspace: for n in [0, N], the sanitised packed start
@@ -66,9 +67,11 @@ WorkspaceLayout tc_workspace_layout(const Problem &p);
 cudaError_t launch_plan(const Problem &p, Plan plan, cudaStream_t stream);
 // T tokens per (sequence, head): q, k, log_alpha [N, T, H, dk], v, o [N, T, H, dv],
 // beta [N, T, H]; S [N, H, dk, dv] read once and written once.
+// gate_per_channel: log_alpha [N, T, H, dk] (1) or [N, T, H] (0).
 cudaError_t launch_decode(const void *q, const void *k, const void *v, kda_dtype_t dt,
                           const float *log_alpha, const float *beta, float *S, int N, int T,
-                          int H, int dk, int dv, float scale, void *o, cudaStream_t stream);
+                          int H, int dk, int dv, float scale, void *o, int gate_per_channel,
+                          cudaStream_t stream);
 // Prefill phases: bit 0 = prepare (plan + chunk-parallel kernel), bit 1 = carry.
 enum : int { kPhasePrepare = 1, kPhaseCarry = 2, kPhaseAll = 3 };
 cudaError_t launch_simt_prefill(const Problem &p, void *workspace, int phases,

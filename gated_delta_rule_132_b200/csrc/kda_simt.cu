@@ -39,6 +39,7 @@ struct SimtParams {
     const void *q, *k, *v;
     const float *log_alpha, *beta, *S0;
     int N, H;
+    int gate_per_channel;  // log_alpha [.., H, D] (1) or [.., H] (0)
     float scale;
     void *o;
     float *S_final;
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1) simt_prep_kernel(SimtParams p
         if (r < L) {
             const size_t off = ((size_t)(t0 + r) * H + h) * D + i;
             kq = to_f32(k[off]); qq = to_f32(q[off]); vv = to_f32(v[off]);
-            la = p.log_alpha[off];
+            la = p.gate_per_channel ? p.log_alpha[off] : p.log_alpha[(size_t)(t0 + r) * H + h];
         }
         sk[r * DP + i] = kq; sq[r * DP + i] = qq; sv[r * D + i] = vv; sg[r * DP + i] = la;
     }
@@ -269,6 +270,7 @@ cudaError_t launch_simt_d(const Problem &pb, void *workspace, int phases, cudaSt
     p.q = pb.q; p.k = pb.k; p.v = pb.v;
     p.log_alpha = pb.log_alpha; p.beta = pb.beta; p.S0 = pb.S0;
     p.N = pb.N; p.H = pb.H; p.scale = pb.scale; p.o = pb.o; p.S_final = pb.S_final;
+    p.gate_per_channel = pb.gate_per_channel;
     Plan plan;
     plan.seq_start = static_cast<int32_t *>(workspace);
     plan.chunk_off = plan.seq_start + (pb.N + 1);

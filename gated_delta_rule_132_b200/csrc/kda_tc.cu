@@ -285,6 +285,83 @@ __device__ __forceinline__ void strip_dot(const float *X, int xr, int xc, const 
 
 __device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y, -v.z, -v.w); }
 
+// T = (I + A)^{-1} for the 64x64 strictly lower A (fp32, row stride kLd), by
+// blocks of 16 on 256 threads: the four diagonal blocks by substitution, then
+// the off-diagonal blocks by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
+// Ts (row stride kLd) receives the blocks on and below the diagonal; the
+// blocks above it are not written. Ys is 3 x 16 x 16 fp32 scratch. Ends with a
+// CTA barrier.
+__device__ __forceinline__ void invert_unit_lower64(const float *As, float *Ts, float *Ys, int tid)
+{
+    if (tid < 64) {  // diagonal blocks: one column of one block per thread, right-looking
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 15; ++s2) {
+            float col[15];
+#pragma unroll
+            for (int r = s2 + 1; r < 16; ++r) col[r - 1] = As[(o + r) * kLd + o + s2];
+            const float xs = x[s2];
+#pragma unroll
+            for (int r = s2 + 1; r < 16; ++r) x[r] -= col[r - 1] * xs;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ts[(o + r) * kLd + o + cc] = x[r];
+    }
+    __syncthreads();
+    // Off-diagonal blocks by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, in
+    // 1x4 strips: thread -> (block, row rr, column group c4).
+    const int rr = (tid & 63) >> 2, c4 = tid & 3, blk = tid >> 6;
+    // distance 1: i = 1..3 on threads 0..191
+    if (blk < 3) {
+        const int i = 1 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), kLd, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ys + blk * 256 + rr * 16 + 4 * c4) = acc;
+    }
+    __syncthreads();
+    if (blk < 3) {
+        const int i = 1 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(Ts, 16 * i, 16 * i, Ys + blk * 256, 0, 0, 16, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ts + (16 * i + rr) * kLd + 16 * (i - 1) + 4 * c4) = neg4(acc);
+    }
+    __syncthreads();
+    // distance 2: i = 2, 3 on threads 0..127
+    if (blk < 2) {
+        const int i = 2 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), kLd, rr, c4, acc);
+        strip_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), kLd, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ys + blk * 256 + rr * 16 + 4 * c4) = acc;
+    }
+    __syncthreads();
+    if (blk < 2) {
+        const int i = 2 + blk;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(Ts, 16 * i, 16 * i, Ys + blk * 256, 0, 0, 16, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ts + (16 * i + rr) * kLd + 16 * (i - 2) + 4 * c4) = neg4(acc);
+    }
+    __syncthreads();
+    // distance 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20) on threads 0..63
+    if (blk == 0) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(As, 48, 0, Ts, 0, 0, kLd, rr, c4, acc);
+        strip_dot(As, 48, 16, Ts, 16, 0, kLd, rr, c4, acc);
+        strip_dot(As, 48, 32, Ts, 32, 0, kLd, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ys + rr * 16 + 4 * c4) = acc;
+    }
+    __syncthreads();
+    if (blk == 0) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        strip_dot(Ts, 48, 48, Ys, 0, 0, 16, rr, c4, acc);
+        *reinterpret_cast<float4 *>(Ts + (48 + rr) * kLd + 4 * c4) = neg4(acc);
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -576,73 +653,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         uint4 *z = reinterpret_cast<uint4 *>(sm + Prep2Smem::kTt + 8192);
         for (int i = tid; i < 8192 / 16; i += kPrep2Threads) z[i] = make_uint4(0, 0, 0, 0);
     }
-    if (tid < 64) {  // diagonal blocks: one column of one block per thread, right-looking
-        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < 15; ++s2) {
-            float col[15];
-#pragma unroll
-            for (int r = s2 + 1; r < 16; ++r) col[r - 1] = As[(o + r) * kLd + o + s2];
-            const float xs = x[s2];
-#pragma unroll
-            for (int r = s2 + 1; r < 16; ++r) x[r] -= col[r - 1] * xs;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Ts[(o + r) * kLd + o + cc] = x[r];
-    }
-    __syncthreads();
-    // Off-diagonal blocks by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, in
-    // 1x4 strips: thread -> (block, row rr, column group c4).
-    const int rr = (tid & 63) >> 2, c4 = tid & 3, blk = tid >> 6;
-    // distance 1: i = 1..3 on threads 0..191
-    if (blk < 3) {
-        const int i = 1 + blk;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        strip_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 1), kLd, rr, c4, acc);
-        *reinterpret_cast<float4 *>(Ys + blk * 256 + rr * 16 + 4 * c4) = acc;
-    }
-    __syncthreads();
-    if (blk < 3) {
-        const int i = 1 + blk;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        strip_dot(Ts, 16 * i, 16 * i, Ys + blk * 256, 0, 0, 16, rr, c4, acc);
-        *reinterpret_cast<float4 *>(Ts + (16 * i + rr) * kLd + 16 * (i - 1) + 4 * c4) = neg4(acc);
-    }
-    __syncthreads();
-    // distance 2: i = 2, 3 on threads 0..127
-    if (blk < 2) {
-        const int i = 2 + blk;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        strip_dot(As, 16 * i, 16 * (i - 2), Ts, 16 * (i - 2), 16 * (i - 2), kLd, rr, c4, acc);
-        strip_dot(As, 16 * i, 16 * (i - 1), Ts, 16 * (i - 1), 16 * (i - 2), kLd, rr, c4, acc);
-        *reinterpret_cast<float4 *>(Ys + blk * 256 + rr * 16 + 4 * c4) = acc;
-    }
-    __syncthreads();
-    if (blk < 2) {
-        const int i = 2 + blk;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        strip_dot(Ts, 16 * i, 16 * i, Ys + blk * 256, 0, 0, 16, rr, c4, acc);
-        *reinterpret_cast<float4 *>(Ts + (16 * i + rr) * kLd + 16 * (i - 2) + 4 * c4) = neg4(acc);
-    }
-    __syncthreads();
-    // distance 3: T_30 = -T_33 (A_30 T_00 + A_31 T_10 + A_32 T_20) on threads 0..63
-    if (blk == 0) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        strip_dot(As, 48, 0, Ts, 0, 0, kLd, rr, c4, acc);
-        strip_dot(As, 48, 16, Ts, 16, 0, kLd, rr, c4, acc);
-        strip_dot(As, 48, 32, Ts, 32, 0, kLd, rr, c4, acc);
-        *reinterpret_cast<float4 *>(Ys + rr * 16 + 4 * c4) = acc;
-    }
-    __syncthreads();
-    if (blk == 0) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        strip_dot(Ts, 48, 48, Ys, 0, 0, 16, rr, c4, acc);
-        *reinterpret_cast<float4 *>(Ts + (48 + rr) * kLd + 4 * c4) = neg4(acc);
-    }
-    __syncthreads();
+    invert_unit_lower64(As, Ts, Ys, tid);
     {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
         uint8_t *tt = sm + Prep2Smem::kTt;
@@ -689,6 +700,274 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         tc::tc_fence_after_sync();
         const int lg = warp & 3, wh = warp >> 2;
         const int row = lg * 32 + (tid & 31);
+        const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
+        float w[32];
+        if (lg < 2) {
+            uint8_t *a1 = rec + Record::kA1 + (uint32_t)wh * 16384;
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
+                    *reinterpret_cast<uint4 *>(a1 + tc::sw128(row, (q2 * 4 + c16) * 16)) =
+                        make_uint4(u[0], u[1], u[2], u[3]);
+                }
+            }
+        }
+        tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
+        uint8_t *uu = rec + Record::kU + (uint32_t)(row >> 6) * 16384;
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            *reinterpret_cast<float4 *>(uu + u_swz(row & 63, 32 * wh + 4 * m)) =
+                make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+    }
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after_sync();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+// ------------------------------------------------------------------- GDN prep
+// Gate shared by all channels (one log-decay per token and head, the gated
+// DeltaNet case of the rule). With g_r the chunk's inclusive cumulative
+// log-decay, every decay factor of A and P is e^{g_r - g_s} <= 1 (s <= r) and
+// comes out of the channel contraction, so
+//     A_rs = beta_r e^{g_r - g_s} (K K^T)_rs  (s < r),   P_rs = e^{g_r - g_s} (Q K^T)_rs  (s <= r)
+// come from one MMA on the raw bf16 tiles, D (128x64) = [K; Q] . K^T, scaled in
+// the epilogue: no reference tokens and no fixup. The diagonal scalings of the
+// solve fold into T: W = (T Diag(beta e^g)) K and U~^T = V^T (T Diag(beta))^T.
+// The record is the one the carry kernel reads for per-channel gates, with
+// gamma = e^{g_C} in every channel. One CTA per (chunk, head), 256 threads.
+constexpr int kGdnThreads = 256;
+
+struct GdnSmem {
+    static constexpr uint32_t kQK = 0;        // 32768: [K; Q] bf16, K-major SW128, 2 K-blocks x 128 rows
+    static constexpr uint32_t kV = 32768;     // 16384: V bf16, [channel block][64 tokens][128 B] SW128
+    static constexpr uint32_t kA = 49152;     // fp32 A [64][kLd]
+    static constexpr uint32_t kT = 66560;     // fp32 T [64][kLd]
+    static constexpr uint32_t kY = 83968;     // fp32 3 x [16][16] block products
+    static constexpr uint32_t kTw = 87040;    // 16384: [T Diag(beta e^g); 0] bf16, K-major rows r
+    static constexpr uint32_t kTu = 103424;   // 8192:  T Diag(beta) bf16, K-major rows r
+    static constexpr uint32_t kG = 111616;    // fp32 g [64], beta [64]
+    static constexpr uint32_t kBar = 112128;  // barriers + tmem slot + flags
+    static constexpr uint32_t kBytes = kBar + 64 + 1024;
+};
+static_assert(GdnSmem::kA == GdnSmem::kV + 16384 && GdnSmem::kT == GdnSmem::kA + 64 * kLd * 4 &&
+              GdnSmem::kY == GdnSmem::kT + 64 * kLd * 4 && GdnSmem::kTw >= GdnSmem::kY + 3072 &&
+              GdnSmem::kTw % 1024 == 0 && GdnSmem::kTu % 1024 == 0 &&
+              GdnSmem::kG == GdnSmem::kTu + 8192, "GDN prep layout");
+
+// 8 bf16 values times one fp32 factor, rounded once.
+__device__ __forceinline__ uint4 scale8(uint4 x, float f)
+{
+    const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(f * __low2float(x2[j]), f * __high2float(x2[j]));
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar_ap = reinterpret_cast<uint64_t *>(sm + GdnSmem::kBar);
+    uint64_t *bar_wu = bar_ap + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ap + 2);
+    volatile int *abort = reinterpret_cast<volatile int *>(bar_ap + 3);
+    float *sg = reinterpret_cast<float *>(sm + GdnSmem::kG);
+    float *sbeta = sg + C;
+
+    const int c = blockIdx.x, h = blockIdx.y, H = p.H;
+    const int n = find_seq(p.chunk_off, p.N, c);
+    if (n < 0) return;  // uniform over the CTA: nothing allocated yet
+    const int t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
+    const int L = min(C, p.seq_start[n + 1] - t0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        tc::mbar_init(bar_ap, 1);
+        tc::mbar_init(bar_wu, 1);
+        *abort = 0;
+        tc::fence_mbar_init();
+    }
+    // ---- 1. k, q, v straight into their operand layouts, 16-byte granules
+    // (thread -> token row r, channel octet oc), rows past the chunk's end zero
+#pragma unroll
+    for (int j = 0; j < 12; ++j) {
+        const int gi = tid + kGdnThreads * j;
+        const int sel = gi >> 10, r = (gi >> 4) & 63, oc = gi & 15;  // sel: k, q, v
+        const uint32_t kb = (uint32_t)(oc >> 3), sw = (uint32_t)(((oc & 7) ^ (r & 7)) << 4);
+        uint8_t *dst = sel == 2 ? sm + GdnSmem::kV + kb * 8192 + r * 128 + sw
+                                : sm + GdnSmem::kQK + kb * 16384 + (sel * 64 + r) * 128 + sw;
+        if (r < L) {
+            const __nv_bfloat16 *src = sel == 0 ? p.k : (sel == 1 ? p.q : p.v);
+            tc::cp_async16(dst, src + ((size_t)(t0 + r) * H + h) * D + 8 * oc);
+        } else {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    if (warp == 0) { tc::tmem_alloc(tmem_slot, 256); tc::tmem_relinquish(); }
+    if (warp == 1) {
+        // inclusive cumulative log-decay of the 64 tokens, two per lane
+        const int r0 = 2 * lane, r1 = r0 + 1;
+        const float a0 = r0 < L ? p.log_alpha[(size_t)(t0 + r0) * H + h] : 0.f;
+        const float a1 = r1 < L ? p.log_alpha[(size_t)(t0 + r1) * H + h] : 0.f;
+        float run = a0 + a1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, run, off);
+            if (lane >= off) run += y;
+        }
+        sg[r1] = run;
+        sg[r0] = run - a1;
+    } else if (warp == 2) {
+        for (int r = lane; r < C; r += 32) sbeta[r] = r < L ? p.beta[(size_t)(t0 + r) * H + h] : 0.f;
+    }
+    tc::cp_async_wait_all();
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    tc::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- 2. D (128x64) = [K; Q] . K^T: rows 0..63 K K^T, rows 64..127 Q K^T
+    if (tid == 0) {
+        const uint32_t a0 = tc::smem_u32(sm + GdnSmem::kQK);
+        const uint32_t id = tc::idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = tc::smem_desc(a0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(tmem, d, d, id, kk > 0);  // B = the K rows (the first 64) of A
+        }
+        tc::mma_commit(bar_ap);
+    }
+    // ---- 3. record pieces that need only the gates, while the MMA runs:
+    // Q~ = e^{g_r} q_r (rows 64.. of [W; Q~]), K^ = e^{g_C - g_s} k_s, gamma
+    uint8_t *rec = p.rec + ((size_t)c * H + h) * Record::kBytes;
+    const float gC = sg[C - 1];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int gi = tid + kGdnThreads * j;
+        const int sel = gi >> 10, r = (gi >> 4) & 63, oc = gi & 15;  // sel: k, q
+        const uint32_t kb = (uint32_t)(oc >> 3), sw = (uint32_t)(((oc & 7) ^ (r & 7)) << 4);
+        const uint4 x = *reinterpret_cast<const uint4 *>(sm + GdnSmem::kQK + kb * 16384 +
+                                                        (sel * 64 + r) * 128 + sw);
+        if (sel == 0)
+            *reinterpret_cast<uint4 *>(rec + Record::kKh + kb * 8192 + r * 128 + sw) =
+                scale8(x, __expf(gC - sg[r]));
+        else
+            *reinterpret_cast<uint4 *>(rec + Record::kA1 + kb * 16384 + (64 + r) * 128 + sw) =
+                scale8(x, __expf(sg[r]));
+    }
+    if (tid < D) reinterpret_cast<float *>(rec + Record::kG)[tid] = __expf(gC);
+
+    // ---- 4. A (fp32, strictly lower, beta-scaled) and P (record) from D
+    float *As = reinterpret_cast<float *>(sm + GdnSmem::kA);
+    float *Ts = reinterpret_cast<float *>(sm + GdnSmem::kT);
+    float *Ys = reinterpret_cast<float *>(sm + GdnSmem::kY);
+    {
+        tc::mbar_wait(bar_ap, 0, abort, p.err, 21);
+        tc::tc_fence_after_sync();
+        const int t = (warp & 3) * 32 + lane;  // accumulator row
+        const int sh = (warp >> 2) * 32;       // first column s of this thread
+        float d[32];
+        tc::tmem_ld32_sync(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)sh, d);
+        if (t < C) {
+            const int r = t;
+            const float gr = sg[r], b = sbeta[r];
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                float v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int s2 = sh + e + q;
+                    v[q] = s2 < r ? b * __expf(gr - sg[s2]) * d[e + q] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(As + r * kLd + sh + e) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+        } else {
+            const int r = t - C;
+            const float gr = sg[r];
+            uint8_t *prow = rec + Record::kP;
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int s0 = sh + c16 * 8 + 2 * e;
+                    w[e] = pack_bf16x2(s0 <= r ? __expf(gr - sg[s0]) * d[c16 * 8 + 2 * e] : 0.f,
+                                       s0 + 1 <= r ? __expf(gr - sg[s0 + 1]) * d[c16 * 8 + 2 * e + 1] : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(prow + tc::sw128(r, (sh / 8 + c16) * 16)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+    tc::tc_fence_before_sync();
+    __syncthreads();
+
+    // ---- 5. T = (I + A)^{-1}, then the two scaled T images
+    {   // rows 64..127 of [T Diag(beta e^g); 0] are zero
+        uint4 *z = reinterpret_cast<uint4 *>(sm + GdnSmem::kTw + 8192);
+        for (int i = tid; i < 8192 / 16; i += kGdnThreads) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    invert_unit_lower64(As, Ts, Ys, tid);
+    {
+        const int r = tid >> 2, s0 = (tid & 3) * 16;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t ww[4], wu[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int sa = s0 + h2 * 8 + 2 * e, sb2 = sa + 1;
+                const float ta = sa < r ? Ts[r * kLd + sa] : (sa == r ? 1.f : 0.f);
+                const float tb = sb2 < r ? Ts[r * kLd + sb2] : (sb2 == r ? 1.f : 0.f);
+                const float ba = sbeta[sa] * ta, bb = sbeta[sb2] * tb;
+                wu[e] = pack_bf16x2(ba, bb);
+                ww[e] = pack_bf16x2(ba * __expf(sg[sa]), bb * __expf(sg[sb2]));
+            }
+            const uint32_t off = tc::sw128(r, (s0 + h2 * 8) * 2);
+            *reinterpret_cast<uint4 *>(sm + GdnSmem::kTw + off) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+            *reinterpret_cast<uint4 *>(sm + GdnSmem::kTu + off) = make_uint4(wu[0], wu[1], wu[2], wu[3]);
+        }
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    tc::tc_fence_after_sync();
+
+    // ---- 6. W = [T Diag(beta e^g); 0] . K and U~^T = V^T . (T Diag(beta))^T
+    if (tid == 0) {
+        const uint32_t kq = tc::smem_u32(sm + GdnSmem::kQK);  // K rows as MN-major B: atoms 16 KB apart
+        const uint32_t vv = tc::smem_u32(sm + GdnSmem::kV);
+        const uint32_t tw = tc::smem_u32(sm + GdnSmem::kTw);
+        const uint32_t tu = tc::smem_u32(sm + GdnSmem::kTu);
+        const uint32_t idw = tc::idesc_bf16(128, 128, 0, 1);
+        const uint32_t idu = tc::idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem, tc::smem_desc(tw + kk * 32, 16, 1024),
+                         tc::smem_desc(kq + kk * 2048, 16384, 1024), idw, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem + 128, tc::smem_desc(vv + kk * 2048, 8192, 1024),
+                         tc::smem_desc(tu + kk * 32, 16, 1024), idu, kk > 0);
+        tc::mma_commit(bar_wu);
+    }
+    {
+        // W: lanes 0..63 (tokens), columns 0..127 (channels 64*wh..): warps 0,1,4,5.
+        // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
+        tc::mbar_wait(bar_wu, 0, abort, p.err, 22);
+        tc::tc_fence_after_sync();
+        const int lg = warp & 3, wh = warp >> 2;
+        const int row = lg * 32 + lane;
         const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
         float w[32];
         if (lg < 2) {
@@ -1036,7 +1315,14 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
         if (e != cudaSuccess) return e;
         e = cudaMemsetAsync(p.err, 0, 2 * sizeof(int), st);
         if (e != cudaSuccess) return e;
-        if (pb.max_chunks > 0) {
+        if (pb.max_chunks > 0 && !pb.gate_per_channel) {
+            e = cudaFuncSetAttribute(tc_gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)GdnSmem::kBytes);
+            if (e != cudaSuccess) return e;
+            tc_gdn_prep_kernel<<<dim3(pb.max_chunks, pb.H), kGdnThreads, GdnSmem::kBytes, st>>>(p);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        } else if (pb.max_chunks > 0) {
             e = cudaFuncSetAttribute(tc_prep2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)Prep2Smem::kBytes);
             if (e != cudaSuccess) return e;

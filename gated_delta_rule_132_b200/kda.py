@@ -59,15 +59,17 @@ def lib() -> ctypes.CDLL:
                   _vp, _vp, _vp, _sz]
         L.kda_chunk_fwd.restype = _i
         L.kda_chunk_fwd.argtypes = common + [_vp]
-        for fn in ("kda_chunk_fwd_ex", "kda_chunk_fwd_prepare", "kda_chunk_fwd_carry"):
+        for fn in ("kda_chunk_fwd_ex", "kda_chunk_fwd_prepare", "kda_chunk_fwd_carry",
+                   "kda_gdn_chunk_fwd", "kda_gdn_chunk_fwd_prepare"):
             getattr(L, fn).restype = _i
             getattr(L, fn).argtypes = common + [_i, _vp]
         L.kda_decode_step.restype = _i
         L.kda_decode_step.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                                       _vp, _vp]
-        L.kda_decode_tokens.restype = _i
-        L.kda_decode_tokens.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i,
-                                        _f, _vp, _vp]
+        for fn in ("kda_decode_tokens", "kda_gdn_decode_tokens"):
+            getattr(L, fn).restype = _i
+            getattr(L, fn).argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                       _f, _vp, _vp]
         _lib = L
     return _lib
 
@@ -112,11 +114,16 @@ class ChunkFwdCall:
     """One prefill problem marshalled for the C ABI: the checked tensors, the
     outputs, the workspace and the ctypes argument list. Calling ``run``,
     ``prepare`` or ``carry`` enqueues ``kda_chunk_fwd_ex`` or one of its two
-    phases on ``stream`` (default: the current torch stream)."""
+    phases on ``stream`` (default: the current torch stream). With
+    ``gate="head"`` log_alpha is [B,T,H] (one gate per head, the GDN entry
+    points ``kda_gdn_chunk_fwd`` and ``kda_gdn_chunk_fwd_prepare``)."""
 
     def __init__(self, q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None,
                  output_final_state=True, workspace=None, o=None, S_final=None,
-                 algo="auto"):
+                 algo="auto", gate="channel"):
+        if gate not in ("channel", "head"):
+            raise ValueError(f"gate must be 'channel' or 'head', not {gate!r}")
+        self.gate = gate
         B, T, H, dk = q.shape
         dv = v.shape[-1]
         dtype = q.dtype
@@ -124,7 +131,8 @@ class ChunkFwdCall:
         for t, name in ((q, "q"), (k, "k")):
             _need(t, name, dtype, (B, T, H, dk))
         _need(v, "v", dtype, (B, T, H, dv))
-        _need(log_alpha, "log_alpha", torch.float32, (B, T, H, dk))
+        _need(log_alpha, "log_alpha", torch.float32,
+              (B, T, H, dk) if gate == "channel" else (B, T, H))
         _need(beta, "beta", torch.float32, (B, T, H))
         if cu_seqlens is not None:
             _need(cu_seqlens, "cu_seqlens", torch.int32)
@@ -161,10 +169,12 @@ class ChunkFwdCall:
         return self.o, self.S_final
 
     def run(self, stream=None):
-        return self._call("kda_chunk_fwd_ex", stream)
+        return self._call("kda_chunk_fwd_ex" if self.gate == "channel" else "kda_gdn_chunk_fwd",
+                          stream)
 
     def prepare(self, stream=None):
-        return self._call("kda_chunk_fwd_prepare", stream)
+        return self._call("kda_chunk_fwd_prepare" if self.gate == "channel"
+                          else "kda_gdn_chunk_fwd_prepare", stream)
 
     def carry(self, stream=None):
         return self._call("kda_chunk_fwd_carry", stream)
@@ -197,6 +207,17 @@ def kda_chunk_fwd_carry(call: ChunkFwdCall, stream=None):
     return call.carry(stream)
 
 
+def kda_gdn_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None,
+                      output_final_state=True, workspace=None, o=None, S_final=None,
+                      algo="auto", stream=None):
+    """Chunked prefill with one gate per token and head (C: ``kda_gdn_chunk_fwd``).
+
+    As :func:`kda_chunk_fwd`, except log_alpha is [B,T,H] fp32.
+    """
+    return ChunkFwdCall(q, k, v, log_alpha, beta, S0, cu_seqlens, scale, output_final_state,
+                        workspace, o, S_final, algo, gate="head").run(stream)
+
+
 def kda_decode_step(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None):
     """One recurrent decode step (C: ``kda_decode_step``); updates S in place.
 
@@ -226,11 +247,13 @@ def kda_decode_step(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None
     return o
 
 
-def kda_decode_tokens(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None):
+def kda_decode_tokens(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None,
+                      gate="channel"):
     """T recurrent decode steps in one call (C: ``kda_decode_tokens``); updates S in place.
 
-    q, k [N,T,H,dk]; v [N,T,H,dv] (bf16 or fp32); log_alpha [N,T,H,dk] fp32;
-    beta [N,T,H] fp32; S [N,H,dk,dv] fp32. Returns o [N,T,H,dv] in q's dtype.
+    q, k [N,T,H,dk]; v [N,T,H,dv] (bf16 or fp32); log_alpha [N,T,H,dk] fp32
+    ([N,T,H] with ``gate="head"``, C: ``kda_gdn_decode_tokens``); beta [N,T,H]
+    fp32; S [N,H,dk,dv] fp32. Returns o [N,T,H,dv] in q's dtype.
     """
     N, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -239,7 +262,10 @@ def kda_decode_tokens(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=No
     _need(q, "q", dtype, (N, T, H, dk))
     _need(k, "k", dtype, (N, T, H, dk))
     _need(v, "v", dtype, (N, T, H, dv))
-    _need(log_alpha, "log_alpha", torch.float32, (N, T, H, dk))
+    if gate not in ("channel", "head"):
+        raise ValueError(f"gate must be 'channel' or 'head', not {gate!r}")
+    _need(log_alpha, "log_alpha", torch.float32,
+          (N, T, H, dk) if gate == "channel" else (N, T, H))
     _need(beta, "beta", torch.float32, (N, T, H))
     _need(S, "S", torch.float32, (N, H, dk, dv))
     if scale is None:
@@ -248,8 +274,9 @@ def kda_decode_tokens(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=No
         o = torch.empty((N, T, H, dv), dtype=dtype, device=q.device)
     else:
         _need(o, "o", dtype, (N, T, H, dv))
-    st = lib().kda_decode_tokens(_p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S),
-                                 N, T, H, dk, dv, float(scale), _p(o), _stream(stream))
+    fn = "kda_decode_tokens" if gate == "channel" else "kda_gdn_decode_tokens"
+    st = getattr(lib(), fn)(_p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S),
+                            N, T, H, dk, dv, float(scale), _p(o), _stream(stream))
     if st != 0:
-        raise KdaError("kda_decode_tokens", st)
+        raise KdaError(fn, st)
     return o

@@ -188,6 +188,46 @@ kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v,
                                int dv, float scale, void *o, void *stream);
 
 /*
+ * Gated DeltaNet (GDN) variants: the same update rule with one forget rate per
+ * token and head instead of one per channel, i.e. Diag(alpha_t) = alpha_t I.
+ * Source: "Kimi Linear：让长上下文大模型真正实用的线性注意力架构" (juejin.cn),
+ * section 三 1️⃣ (GDN has a single forget rate per head; KDA refines it per
+ * channel) with the rule of section 三 5️⃣. Results equal the KDA entry points
+ * given log_alpha broadcast over the dk channels.
+ *
+ * kda_gdn_chunk_fwd: arguments, layouts, workspace (kda_chunk_fwd_workspace_size_ex
+ * with the same algo), errors and paths as kda_chunk_fwd_ex, except
+ *   log_alpha   fp32 [B, T, H]  (one log forget rate per token and head, <= 0)
+ * On the tensor-core path (bf16, dk = dv = 128) the scalar decay comes out of
+ * the channel contraction, so its chunk-parallel phase is a lighter kernel than
+ * the per-channel one; the sequential phase is shared.
+ *
+ * kda_gdn_chunk_fwd_prepare: its chunk-parallel phase alone; the sequential
+ * phase, which reads only the workspace, S0 and the plan, is kda_chunk_fwd_carry
+ * with the same arguments.
+ *
+ * kda_gdn_decode_tokens: as kda_decode_tokens, except
+ *   log_alpha   fp32 [N, T, H]
+ */
+kda_status_t kda_gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                               kda_dtype_t qkv_dtype, const float *log_alpha,
+                               const float *beta, const float *S0, const int32_t *cu_seqlens,
+                               int n_seqs, int B, int T, int H, int dk, int dv, float scale,
+                               void *o, float *S_final, void *workspace,
+                               size_t workspace_bytes, int algo, void *stream);
+kda_status_t kda_gdn_chunk_fwd_prepare(const void *q, const void *k, const void *v,
+                                       kda_dtype_t qkv_dtype, const float *log_alpha,
+                                       const float *beta, const float *S0,
+                                       const int32_t *cu_seqlens, int n_seqs, int B, int T,
+                                       int H, int dk, int dv, float scale, void *o,
+                                       float *S_final, void *workspace, size_t workspace_bytes,
+                                       int algo, void *stream);
+kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v,
+                                   kda_dtype_t qkv_dtype, const float *log_alpha,
+                                   const float *beta, float *S, int N, int T, int H, int dk,
+                                   int dv, float scale, void *o, void *stream);
+
+/*
  * kda_chunk_fwd_noalloc — the chunked prefill for callers that cannot allocate
  * device memory (no counterpart in the paper; it exists for callers such as a
  * plugin whose host application owns all device memory, or code that must not
