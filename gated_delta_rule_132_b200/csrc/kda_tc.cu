@@ -629,7 +629,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
                 *reinterpret_cast<float4 *>(As + r * kLd + sh + e) = make_float4(v[0], v[1], v[2], v[3]);
             }
         } else {
-            uint8_t *prow = rec + Record::kP;
+            uint8_t *prow = sm + Prep2Smem::kTt;  // P staged where [T; 0] goes later
 #pragma unroll
             for (int c16 = 0; c16 < 4; ++c16) {
                 uint32_t w[4];
@@ -644,8 +644,13 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
             }
         }
     }
+    tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
+    if (tid == 0) {
+        tc::bulk_s2g(rec + Record::kP, sm + Prep2Smem::kTt, 8192);
+        tc::bulk_commit();
+    }
 
     // ---- 3. T = (I + A)^{-1} by 16x16 blocks
     {   // rows 64..127 of the [T; 0] operand are zero (this memory held the
@@ -653,6 +658,9 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         uint4 *z = reinterpret_cast<uint4 *>(sm + Prep2Smem::kTt + 8192);
         for (int i = tid; i < 8192 / 16; i += kPrep2Threads) z[i] = make_uint4(0, 0, 0, 0);
     }
+    // the staged P is read before the [T; 0] image overwrites it (the
+    // inverse's barriers order this wait before that)
+    if (tid == 0) tc::bulk_wait_read_all();
     invert_unit_lower64(As, Ts, Ys, tid);
     {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
@@ -696,6 +704,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     {
         // W: lanes 0..63 (tokens), columns 0..127 (channels 64*wh..): warps 0,1,4,5.
         // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
+        // Both as record images in the A / T scratch, dead by now: W rows of
+        // K-block kb at 8K kb, U~^T at 16K.
         tc::mbar_wait(bar_wu, 0, abort, p.err, 12);
         tc::tc_fence_after_sync();
         const int lg = warp & 3, wh = warp >> 2;
@@ -703,7 +713,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
         const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
         float w[32];
         if (lg < 2) {
-            uint8_t *a1 = rec + Record::kA1 + (uint32_t)wh * 16384;
+            uint8_t *a1 = sm + (uint32_t)wh * 8192;
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
@@ -718,14 +728,22 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
             }
         }
         tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
-        uint8_t *uu = rec + Record::kU + (uint32_t)(row >> 6) * 16384;
+        uint8_t *uu = sm + 16384 + (uint32_t)(row >> 6) * 16384;
 #pragma unroll
         for (int m = 0; m < 8; ++m)
             *reinterpret_cast<float4 *>(uu + u_swz(row & 63, 32 * wh + 4 * m)) =
                 make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
     }
+    tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
+    if (tid == 0) {
+        tc::bulk_s2g(rec + Record::kA1, sm, 8192);
+        tc::bulk_s2g(rec + Record::kA1 + 16384, sm + 8192, 8192);
+        tc::bulk_s2g(rec + Record::kU, sm + 16384, 32768);
+        tc::bulk_commit();
+        tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
+    }
     if (warp == 0) {
         tc::tc_fence_after_sync();
         tc::tmem_dealloc(tmem, 256);
@@ -849,8 +867,11 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
         tc::mma_commit(bar_ap);
     }
     // ---- 3. record pieces that need only the gates, while the MMA runs:
-    // Q~ = e^{g_r} q_r (rows 64.. of [W; Q~]), K^ = e^{g_C - g_s} k_s, gamma
+    // K^ = e^{g_C - g_s} k_s and Q~ = e^{g_r} q_r (rows 64.. of [W; Q~]) as their
+    // record images in the (still unused) A/T scratch, sent by bulk copies;
+    // gamma directly. Staging: K^ [0, 16K), Q~ of K-block kb at 16K + 8K kb.
     uint8_t *rec = p.rec + ((size_t)c * H + h) * Record::kBytes;
+    uint8_t *stage = sm + GdnSmem::kA;
     const float gC = sg[C - 1];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -859,14 +880,18 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
         const uint32_t kb = (uint32_t)(oc >> 3), sw = (uint32_t)(((oc & 7) ^ (r & 7)) << 4);
         const uint4 x = *reinterpret_cast<const uint4 *>(sm + GdnSmem::kQK + kb * 16384 +
                                                         (sel * 64 + r) * 128 + sw);
-        if (sel == 0)
-            *reinterpret_cast<uint4 *>(rec + Record::kKh + kb * 8192 + r * 128 + sw) =
-                scale8(x, __expf(gC - sg[r]));
-        else
-            *reinterpret_cast<uint4 *>(rec + Record::kA1 + kb * 16384 + (64 + r) * 128 + sw) =
-                scale8(x, __expf(sg[r]));
+        *reinterpret_cast<uint4 *>(stage + sel * 16384 + kb * 8192 + r * 128 + sw) =
+            scale8(x, __expf(sel == 0 ? gC - sg[r] : sg[r]));
     }
     if (tid < D) reinterpret_cast<float *>(rec + Record::kG)[tid] = __expf(gC);
+    tc::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tc::bulk_s2g(rec + Record::kKh, stage, 16384);
+        tc::bulk_s2g(rec + Record::kA1 + 8192, stage + 16384, 8192);
+        tc::bulk_s2g(rec + Record::kA1 + 16384 + 8192, stage + 16384 + 8192, 8192);
+        tc::bulk_commit();
+    }
 
     // ---- 4. A (fp32, strictly lower, beta-scaled) and P (record) from D
     float *As = reinterpret_cast<float *>(sm + GdnSmem::kA);
@@ -879,6 +904,9 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
         const int sh = (warp >> 2) * 32;       // first column s of this thread
         float d[32];
         tc::tmem_ld32_sync(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)sh, d);
+        // A overwrites the staged K^ / Q~: their bulk copies must have read it
+        if (tid == 0) tc::bulk_wait_read_all();
+        __syncthreads();
         if (t < C) {
             const int r = t;
             const float gr = sg[r], b = sbeta[r];
@@ -895,7 +923,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
         } else {
             const int r = t - C;
             const float gr = sg[r];
-            uint8_t *prow = rec + Record::kP;
+            uint8_t *prow = sm + GdnSmem::kTu;  // P staged where T Diag(beta) goes later
 #pragma unroll
             for (int c16 = 0; c16 < 4; ++c16) {
                 uint32_t w[4];
@@ -910,14 +938,22 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
             }
         }
     }
+    tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
+    if (tid == 0) {
+        tc::bulk_s2g(rec + Record::kP, sm + GdnSmem::kTu, 8192);
+        tc::bulk_commit();
+    }
 
     // ---- 5. T = (I + A)^{-1}, then the two scaled T images
     {   // rows 64..127 of [T Diag(beta e^g); 0] are zero
         uint4 *z = reinterpret_cast<uint4 *>(sm + GdnSmem::kTw + 8192);
         for (int i = tid; i < 8192 / 16; i += kGdnThreads) z[i] = make_uint4(0, 0, 0, 0);
     }
+    // the staged P is read before the T images overwrite it (the inverse's
+    // barriers order this wait before them)
+    if (tid == 0) tc::bulk_wait_read_all();
     invert_unit_lower64(As, Ts, Ys, tid);
     {
         const int r = tid >> 2, s0 = (tid & 3) * 16;
@@ -964,6 +1000,8 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
     {
         // W: lanes 0..63 (tokens), columns 0..127 (channels 64*wh..): warps 0,1,4,5.
         // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
+        // Both as record images in the [K; Q] and V buffers, dead once the MMAs
+        // are done: W rows of K-block kb at 8K kb, U~^T at 16K.
         tc::mbar_wait(bar_wu, 0, abort, p.err, 22);
         tc::tc_fence_after_sync();
         const int lg = warp & 3, wh = warp >> 2;
@@ -971,7 +1009,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
         const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
         float w[32];
         if (lg < 2) {
-            uint8_t *a1 = rec + Record::kA1 + (uint32_t)wh * 16384;
+            uint8_t *a1 = sm + (uint32_t)wh * 8192;
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
@@ -986,14 +1024,22 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
             }
         }
         tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
-        uint8_t *uu = rec + Record::kU + (uint32_t)(row >> 6) * 16384;
+        uint8_t *uu = sm + 16384 + (uint32_t)(row >> 6) * 16384;
 #pragma unroll
         for (int m = 0; m < 8; ++m)
             *reinterpret_cast<float4 *>(uu + u_swz(row & 63, 32 * wh + 4 * m)) =
                 make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
     }
+    tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
+    if (tid == 0) {
+        tc::bulk_s2g(rec + Record::kA1, sm, 8192);
+        tc::bulk_s2g(rec + Record::kA1 + 16384, sm + 8192, 8192);
+        tc::bulk_s2g(rec + Record::kU, sm + 16384, 32768);
+        tc::bulk_commit();
+        tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
+    }
     if (warp == 0) {
         tc::tc_fence_after_sync();
         tc::tmem_dealloc(tmem, 256);

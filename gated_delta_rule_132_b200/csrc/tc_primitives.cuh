@@ -86,6 +86,28 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
                  : "memory");
 }
 
+// Plain bulk copy of this CTA's shared memory to global memory, in the calling
+// thread's current bulk group; commit closes the group. Both addresses 16-byte
+// aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_s2g(void *dst_gmem, const void *src_smem, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst_gmem), "r"(smem_u32(src_smem)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until every bulk group this thread committed has finished reading its
+// shared-memory source (the writes to global memory may still be in flight;
+// they complete before the grid does).
+__device__ __forceinline__ void bulk_wait_read_all()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of
 // this thread's outstanding copies.
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem)
