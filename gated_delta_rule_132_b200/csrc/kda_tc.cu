@@ -26,6 +26,11 @@
 //        MMA3: D1[:, 64:] += U^T . P^T          -> (Q~ S + P U)^T
 //        S^T  = S^T Diag(gamma) + D2;  o = scale * D1[:, 64:]^T
 //    The state never leaves the SM between chunks; S_final is written once.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kda_internal.cuh"
 #include "tc_primitives.cuh"
 
@@ -84,6 +89,10 @@ struct TcParams {
     int *err;          // device error word (pipeline timeouts)
     int *fix_count;    // number of chunks listed for the exact fixup
     int *fix_list;     // chunk * H + head, one per listed chunk
+    // q, k, v and log_alpha as 3-D tensors {channel, head, token} for TMA tile
+    // loads of 128 bytes of channels x 1 head x 64 tokens in the 128-byte
+    // swizzle (64 bf16 or 32 fp32 channels); tm_la only for per-channel gates
+    CUtensorMap tm_q, tm_k, tm_v, tm_la;
 };
 
 __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int c)
@@ -240,7 +249,6 @@ struct Prep2Smem {
     static constexpr uint32_t kA = 0;          // fp32 A [64][kLd], after MMA-AP
     static constexpr uint32_t kBop = 32768;    // 24576: [kb][96 rows][128B]
     static constexpr uint32_t kT = 32768;      // fp32 T [64][kLd], after MMA-AP
-    static constexpr uint32_t kY = 50176;      // fp32 3 x [16][16] block products
     static constexpr uint32_t kBK = 57344;     // 16384: (beta K~) MN-major image
     static constexpr uint32_t kBV = 73728;     // 16384: (beta V) MN-major image (follows BK)
     static constexpr uint32_t kTt = 90112;     // 16384: [T; 0], K-major rows r
@@ -285,13 +293,108 @@ __device__ __forceinline__ void strip_dot(const float *X, int xr, int xc, const 
 
 __device__ __forceinline__ float4 neg4(float4 v) { return make_float4(-v.x, -v.y, -v.z, -v.w); }
 
-// T = (I + A)^{-1} for the 64x64 strictly lower A (fp32, row stride kLd), by
-// blocks of 16 on 256 threads: the four diagonal blocks by substitution, then
-// the off-diagonal blocks by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj.
-// Ts (row stride kLd) receives the blocks on and below the diagonal; the
-// blocks above it are not written. Ys is 3 x 16 x 16 fp32 scratch. Ends with a
-// CTA barrier.
-__device__ __forceinline__ void invert_unit_lower64(const float *As, float *Ts, float *Ys, int tid)
+// T = (I + A)^{-1} for the 64x64 strictly lower A (fp32, row stride kLd) on
+// 256 threads, as a 2x2 block inverse of 32-row blocks whose own inverses are
+// 2x2 block inverses of 16-row blocks: with T_ii the inverses of the four
+// 16x16 diagonal blocks (by substitution),
+//     T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22,
+//     Y = A_[23][01] T_[01][01],  T_[23][01] = -T_[23][23] Y.
+// The 16x16 products are grouped into four phases of up to four independent
+// block tasks (64 threads each, one 1x4 strip per thread); the blocks above
+// T's diagonal, never read by the callers, hold the intermediates:
+//   (0,1) A_10 T_00   (0,2) A_32 T_22   (0,3) Y_21   (1,2) Y_31
+//   (1,3) Y_20        (2,3) Y_30        and T_33 Y_31 sits in (3,1) until T_31.
+// Ts (row stride kLd) receives the blocks on and below the diagonal. Ends with
+// a CTA barrier.
+__device__ __forceinline__ void invert_unit_lower64(const float *As, float *Ts, int tid)
+{
+    if (tid < 64) {  // diagonal blocks: one column of one block per thread, right-looking
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 15; ++s2) {
+            float col[15];
+#pragma unroll
+            for (int r = s2 + 1; r < 16; ++r) col[r - 1] = As[(o + r) * kLd + o + s2];
+            const float xs = x[s2];
+#pragma unroll
+            for (int r = s2 + 1; r < 16; ++r) x[r] -= col[r - 1] * xs;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ts[(o + r) * kLd + o + cc] = x[r];
+    }
+    __syncthreads();
+    const int rr = (tid & 63) >> 2, c4 = tid & 3, task = tid >> 6;
+    auto strip = [&](float *M, int bi, int bj) {  // this thread's 1x4 strip of block (bi, bj)
+        return reinterpret_cast<float4 *>(M + (16 * bi + rr) * kLd + 16 * bj + 4 * c4);
+    };
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    {   // phase 1: A_10 T_00, A_32 T_22, Y_21 = A_21 T_11, Y_31 = A_31 T_11
+        float4 acc = zero;
+        const int ar = task == 0 ? 16 : (task == 1 ? 48 : (task == 2 ? 32 : 48));
+        const int ac = task == 0 ? 0 : (task == 1 ? 32 : 16);
+        strip_dot(As, ar, ac, Ts, ac, ac, kLd, rr, c4, acc);
+        const int sj = task == 3 ? 2 : task + 1, si = task == 3 ? 1 : 0;
+        *strip(Ts, si, sj) = acc;
+    }
+    __syncthreads();
+    {   // phase 2: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22), Y_20, Y_30 = A_[23]0 T_00
+        float4 acc = zero;
+        if (task < 2) {
+            const int d = task == 0 ? 16 : 48;               // T_11 or T_33
+            strip_dot(Ts, d, d, Ts, 0, task == 0 ? 16 : 32, kLd, rr, c4, acc);
+            *strip(Ts, task == 0 ? 1 : 3, task == 0 ? 0 : 2) = neg4(acc);
+        } else {
+            strip_dot(As, task == 2 ? 32 : 48, 0, Ts, 0, 0, kLd, rr, c4, acc);
+            *strip(Ts, task - 1, 3) = acc;                   // (1,3) Y_20, (2,3) Y_30
+        }
+    }
+    __syncthreads();
+    {   // phase 3: Y_20 += A_21 T_10, Y_30 += A_31 T_10, T_21 = -T_22 Y_21, (3,1) = T_33 Y_31
+        if (task < 2) {
+            float4 acc = *strip(Ts, task + 1, 3);
+            strip_dot(As, task == 0 ? 32 : 48, 16, Ts, 16, 0, kLd, rr, c4, acc);
+            *strip(Ts, task + 1, 3) = acc;
+        } else if (task == 2) {
+            float4 acc = zero;
+            strip_dot(Ts, 32, 32, Ts, 0, 48, kLd, rr, c4, acc);
+            *strip(Ts, 2, 1) = neg4(acc);
+        } else {
+            float4 acc = zero;
+            strip_dot(Ts, 48, 48, Ts, 16, 32, kLd, rr, c4, acc);
+            *strip(Ts, 3, 1) = acc;
+        }
+    }
+    __syncthreads();
+    {   // phase 4: T_20 = -T_22 Y_20, T_30 = -(T_32 Y_20 + T_33 Y_30), T_31 = -(T_33 Y_31 + T_32 Y_21)
+        if (task == 0) {
+            float4 acc = zero;
+            strip_dot(Ts, 32, 32, Ts, 16, 48, kLd, rr, c4, acc);
+            *strip(Ts, 2, 0) = neg4(acc);
+        } else if (task == 1) {
+            float4 acc = zero;
+            strip_dot(Ts, 48, 32, Ts, 16, 48, kLd, rr, c4, acc);
+            strip_dot(Ts, 48, 48, Ts, 32, 48, kLd, rr, c4, acc);
+            *strip(Ts, 3, 0) = neg4(acc);
+        } else if (task == 2) {
+            float4 acc = *strip(Ts, 3, 1);
+            strip_dot(Ts, 48, 32, Ts, 0, 48, kLd, rr, c4, acc);
+            *strip(Ts, 3, 1) = neg4(acc);
+        }
+    }
+    __syncthreads();
+}
+
+// The same inverse by block distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj:
+// six phases after the diagonal blocks, with 192, 128 and 64 threads busy at
+// distances 1, 2 and 3 (Ys is 3 x 16 x 16 fp32 scratch). Slower on its own
+// than the grouping above, but the scalar-gate prep, whose two co-resident
+// CTAs fill the idle threads' issue slots, measured faster with it. Ends with
+// a CTA barrier.
+__device__ __forceinline__ void invert_unit_lower64_by_distance(const float *As, float *Ts,
+                                                                float *Ys, int tid)
 {
     if (tid < 64) {  // diagonal blocks: one column of one block per thread, right-looking
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
@@ -362,7 +465,7 @@ __device__ __forceinline__ void invert_unit_lower64(const float *As, float *Ts, 
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
+__global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid_constant__ TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -371,6 +474,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     uint64_t *bar_wu = bar_ap + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ap + 2);
     volatile int *abort = reinterpret_cast<volatile int *>(bar_ap + 3);
+    uint64_t *bar_ld = bar_ap + 4;
     float *tot = reinterpret_cast<float *>(sm + Prep2Smem::kTot);    // [16][128] group totals
     float *cst = reinterpret_cast<float *>(sm + Prep2Smem::kCst);    // [8][128] per channel
     float *sbeta = reinterpret_cast<float *>(sm + Prep2Smem::kB);
@@ -388,29 +492,28 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     const uint32_t kb = (uint32_t)(oc >> 3);   // K-block / MN atom
     const uint32_t ck = (uint32_t)(oc & 7);    // chunk inside the 128-byte row
 
+    // The chunk's q, k, v and log_alpha arrive as ten TMA tiles (64 tokens x
+    // 128 bytes, 128-byte swizzle) in the operand buffers, which step 1 fills
+    // only after every thread holds its inputs in registers: q, k, v as
+    // [channel block of 64][64 tokens][128 B], log_alpha as [block of 32].
+    uint8_t *in_q = sm + Prep2Smem::kAop, *in_k = sm + Prep2Smem::kAop + 16384;
+    uint8_t *in_v = sm + Prep2Smem::kBop, *in_la = sm + Prep2Smem::kBK;
     if (tid == 0) {
         tc::mbar_init(bar_ap, 1);
         tc::mbar_init(bar_wu, 1);
+        tc::mbar_init(bar_ld, 1);
         *abort = 0;
         tc::fence_mbar_init();
-    }
-    // Each thread copies the 16-byte granules it will read (its 8 channels of
-    // q, k, v and log_alpha for its 4 tokens) into the operand buffers, which
-    // step 1 fills only after every thread holds its inputs in registers: the
-    // chunk's 80 KB are in flight at once without holding registers.
-    uint8_t *in_q = sm + Prep2Smem::kAop, *in_k = sm + Prep2Smem::kAop + 16384;
-    uint8_t *in_v = sm + Prep2Smem::kBop, *in_la = sm + Prep2Smem::kBK;
+        tc::mbar_arrive_expect_tx(bar_ld, 10 * 8192);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int r = tg * 4 + e;
-        if (r < L) {
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + c0;
-            tc::cp_async16(in_q + r * 256 + oc * 16, p.q + off);
-            tc::cp_async16(in_k + r * 256 + oc * 16, p.k + off);
-            tc::cp_async16(in_v + r * 256 + oc * 16, p.v + off);
-            tc::cp_async16(in_la + r * 512 + oc * 32, p.log_alpha + off);
-            tc::cp_async16(in_la + r * 512 + oc * 32 + 16, p.log_alpha + off + 4);
+        for (int b = 0; b < 2; ++b) {
+            tc::tma_load_3d(in_q + b * 8192, &p.tm_q, 64 * b, h, t0, bar_ld);
+            tc::tma_load_3d(in_k + b * 8192, &p.tm_k, 64 * b, h, t0, bar_ld);
+            tc::tma_load_3d(in_v + b * 8192, &p.tm_v, 64 * b, h, t0, bar_ld);
         }
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            tc::tma_load_3d(in_la + b * 8192, &p.tm_la, 32 * b, h, t0, bar_ld);
     }
     if (warp == 0) { tc::tmem_alloc(tmem_slot, 256); tc::tmem_relinquish(); }
     if (tid < C) sbeta[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * H + h] : 0.f;
@@ -418,7 +521,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     // ---- 1. loads and the cumulative log-decay
     uint4 qv[4], kv[4], vv[4];
     float g[4][8];
-    tc::cp_async_wait_all();
+    __syncthreads();  // the barriers are initialised
+    tc::mbar_wait(bar_ld, 0, abort, p.err, 10);
     {
         float run[8];
 #pragma unroll
@@ -428,12 +532,14 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
             const int r = tg * 4 + e;
             uint4 q4 = make_uint4(0, 0, 0, 0), k4 = q4, v4 = q4;
             float4 la0 = make_float4(0.f, 0.f, 0.f, 0.f), la1 = la0;
-            if (r < L) {
-                q4 = *reinterpret_cast<const uint4 *>(in_q + r * 256 + oc * 16);
-                k4 = *reinterpret_cast<const uint4 *>(in_k + r * 256 + oc * 16);
-                v4 = *reinterpret_cast<const uint4 *>(in_v + r * 256 + oc * 16);
-                la0 = *reinterpret_cast<const float4 *>(in_la + r * 512 + oc * 32);
-                la1 = *reinterpret_cast<const float4 *>(in_la + r * 512 + oc * 32 + 16);
+            if (r < L) {  // rows past the chunk's end hold the next sequence (or zero)
+                const uint32_t qo = kb * 8192 + r * 128 + ((ck ^ (uint32_t)(r & 7)) << 4);
+                q4 = *reinterpret_cast<const uint4 *>(in_q + qo);
+                k4 = *reinterpret_cast<const uint4 *>(in_k + qo);
+                v4 = *reinterpret_cast<const uint4 *>(in_v + qo);
+                const uint32_t lb = (uint32_t)(oc >> 2) * 8192 + r * 128, j0 = (uint32_t)(oc & 3) * 2;
+                la0 = *reinterpret_cast<const float4 *>(in_la + lb + ((j0 ^ (uint32_t)(r & 7)) << 4));
+                la1 = *reinterpret_cast<const float4 *>(in_la + lb + (((j0 + 1) ^ (uint32_t)(r & 7)) << 4));
             }
             qv[e] = q4; kv[e] = k4; vv[e] = v4;
             run[0] += la0.x; run[1] += la0.y; run[2] += la0.z; run[3] += la0.w;
@@ -602,7 +708,6 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     }
     float *As = reinterpret_cast<float *>(sm + Prep2Smem::kA);   // A[r][s], stride kLd
     float *Ts = reinterpret_cast<float *>(sm + Prep2Smem::kT);   // T[r][s], stride kLd
-    float *Ys = reinterpret_cast<float *>(sm + Prep2Smem::kY);
     {
         // every warp reads its 32 TMEM lanes; warps 0-3 take the first 32 of the
         // row's 64 relevant columns, warps 4-7 the other 32
@@ -661,7 +766,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(TcParams p)
     // the staged P is read before the [T; 0] image overwrites it (the
     // inverse's barriers order this wait before that)
     if (tid == 0) tc::bulk_wait_read_all();
-    invert_unit_lower64(As, Ts, Ys, tid);
+    invert_unit_lower64(As, Ts, tid);
     {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
         uint8_t *tt = sm + Prep2Smem::kTt;
@@ -790,7 +895,7 @@ __device__ __forceinline__ uint4 scale8(uint4 x, float f)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
+__global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __grid_constant__ TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -799,6 +904,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
     uint64_t *bar_wu = bar_ap + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_ap + 2);
     volatile int *abort = reinterpret_cast<volatile int *>(bar_ap + 3);
+    uint64_t *bar_ld = bar_ap + 4;
     float *sg = reinterpret_cast<float *>(sm + GdnSmem::kG);
     float *sbeta = sg + C;
 
@@ -809,26 +915,20 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
     const int L = min(C, p.seq_start[n + 1] - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    // ---- 1. k, q, v straight into their operand layouts: six TMA tiles of 64
+    // channels x 64 tokens (the 128-byte swizzle is the operand swizzle)
     if (tid == 0) {
         tc::mbar_init(bar_ap, 1);
         tc::mbar_init(bar_wu, 1);
+        tc::mbar_init(bar_ld, 1);
         *abort = 0;
         tc::fence_mbar_init();
-    }
-    // ---- 1. k, q, v straight into their operand layouts, 16-byte granules
-    // (thread -> token row r, channel octet oc), rows past the chunk's end zero
+        tc::mbar_arrive_expect_tx(bar_ld, 6 * 8192);
 #pragma unroll
-    for (int j = 0; j < 12; ++j) {
-        const int gi = tid + kGdnThreads * j;
-        const int sel = gi >> 10, r = (gi >> 4) & 63, oc = gi & 15;  // sel: k, q, v
-        const uint32_t kb = (uint32_t)(oc >> 3), sw = (uint32_t)(((oc & 7) ^ (r & 7)) << 4);
-        uint8_t *dst = sel == 2 ? sm + GdnSmem::kV + kb * 8192 + r * 128 + sw
-                                : sm + GdnSmem::kQK + kb * 16384 + (sel * 64 + r) * 128 + sw;
-        if (r < L) {
-            const __nv_bfloat16 *src = sel == 0 ? p.k : (sel == 1 ? p.q : p.v);
-            tc::cp_async16(dst, src + ((size_t)(t0 + r) * H + h) * D + 8 * oc);
-        } else {
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+        for (int kb = 0; kb < 2; ++kb) {
+            tc::tma_load_3d(sm + GdnSmem::kQK + kb * 16384, &p.tm_k, 64 * kb, h, t0, bar_ld);
+            tc::tma_load_3d(sm + GdnSmem::kQK + kb * 16384 + 8192, &p.tm_q, 64 * kb, h, t0, bar_ld);
+            tc::tma_load_3d(sm + GdnSmem::kV + kb * 8192, &p.tm_v, 64 * kb, h, t0, bar_ld);
         }
     }
     if (warp == 0) { tc::tmem_alloc(tmem_slot, 256); tc::tmem_relinquish(); }
@@ -848,7 +948,16 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
     } else if (warp == 2) {
         for (int r = lane; r < C; r += 32) sbeta[r] = r < L ? p.beta[(size_t)(t0 + r) * H + h] : 0.f;
     }
-    tc::cp_async_wait_all();
+    // rows past the chunk's end (the next sequence, or past the tensor) read zero
+    __syncthreads();  // the barriers are initialised
+    tc::mbar_wait(bar_ld, 0, abort, p.err, 20);
+    for (int i = tid; i < 6 * (C - L) * 8; i += kGdnThreads) {
+        const int tile = i / ((C - L) * 8), rem = i % ((C - L) * 8);
+        const int r = L + (rem >> 3);
+        uint8_t *base = tile < 4 ? sm + GdnSmem::kQK + (tile >> 1) * 16384 + (tile & 1) * 8192
+                                 : sm + GdnSmem::kV + (tile - 4) * 8192;
+        *reinterpret_cast<uint4 *>(base + r * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+    }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before_sync();
     __syncthreads();
@@ -954,7 +1063,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(TcParams p)
     // the staged P is read before the T images overwrite it (the inverse's
     // barriers order this wait before them)
     if (tid == 0) tc::bulk_wait_read_all();
-    invert_unit_lower64(As, Ts, Ys, tid);
+    invert_unit_lower64_by_distance(As, Ts, Ys, tid);
     {
         const int r = tid >> 2, s0 = (tid & 3) * 16;
 #pragma unroll
@@ -1319,6 +1428,41 @@ constexpr int kFixupBlocks = 148;
 
 }  // namespace
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link to the
+// driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// [tokens, H, 128] (bf16 or fp32) as a {128, H, tokens} tensor with boxes of
+// 128 bytes of channels x 1 head x 64 tokens in the 128-byte swizzle;
+// out-of-range tokens read zero.
+bool encode_token_map(CUtensorMap *tm, const void *base, bool fp32, int H, long long tokens)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t es = fp32 ? 4 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / es), 1, (cuuint32_t)C};
+    cuuint32_t estride[3] = {1, 1, 1};
+    return enc(tm, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void *>(base), dims, strides, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 bool tc_supported(const Problem &p)
 {
     return p.dtype == KDA_DTYPE_BF16 && p.dk == 128 && p.dv == 128;
@@ -1361,6 +1505,13 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
         if (e != cudaSuccess) return e;
         e = cudaMemsetAsync(p.err, 0, 2 * sizeof(int), st);
         if (e != cudaSuccess) return e;
+        if (pb.max_chunks > 0 &&
+            (!encode_token_map(&p.tm_q, pb.q, false, pb.H, pb.total_tokens) ||
+             !encode_token_map(&p.tm_k, pb.k, false, pb.H, pb.total_tokens) ||
+             !encode_token_map(&p.tm_v, pb.v, false, pb.H, pb.total_tokens) ||
+             (pb.gate_per_channel &&
+              !encode_token_map(&p.tm_la, pb.log_alpha, true, pb.H, pb.total_tokens))))
+            return cudaErrorInvalidValue;
         if (pb.max_chunks > 0 && !pb.gate_per_channel) {
             e = cudaFuncSetAttribute(tc_gdn_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)GdnSmem::kBytes);

@@ -86,6 +86,20 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
                  : "memory");
 }
 
+// 3-D tiled tensor copy (TMA) global -> this CTA's shared memory, completing
+// its bytes on an mbarrier; no multicast. `tmap` is the generic address of a
+// CUtensorMap in kernel-parameter space (a __grid_constant__ argument);
+// coordinates innermost first. The innermost coordinate times the element
+// size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tmap, int x, int y, int z,
+                                            uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3, %4}], [%5];"
+                 ::"r"(smem_u32(dst_smem)), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // Plain bulk copy of this CTA's shared memory to global memory, in the calling
 // thread's current bulk group; commit closes the group. Both addresses 16-byte
 // aligned, size a multiple of 16.
