@@ -42,9 +42,10 @@ LAUNCHES_PER_PREFILL = 4
 # DRAM traffic per (chunk, head) record measured by ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum) on the chunked workload, one launch of 4096 records;
 # traffic grows in proportion to the records a launch processes. Sources:
-# profiles/tc_prep2_kernel_chunked_B4_H16_T4096.md and
+# profiles/tc_prep2_kernel_chunked_B4_H16_T4096.md,
+# profiles/tc_gdn_prep_kernel_chunked_B4_H16_T4096.md and
 # profiles/tc_carry_kernel_chunked_B4_H16_T4096.md.
-TRAFFIC_PER_RECORD = {"prepare": 162_304, "carry": 105_469}
+TRAFFIC_PER_RECORD = {"prepare": 162_115, "carry": 105_452, "gdn_prepare": 128_435}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -447,7 +448,8 @@ def run_ours(args, world, rank, dev):
             "kernels_ms": {"prepare": round(gdn["prep_ms"], 4), "carry": round(gdn["carry_ms"], 4)},
             "roofline": {"kernel": "prepare (one gate per head)", "bound": "hbm",
                          "achieved": round(g_ach, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(g_ach / hbm, 4), "traffic": None,
+                         "frac": round(g_ach / hbm, 4),
+                         "traffic": TRAFFIC_PER_RECORD["gdn_prepare"] * pre["records"],
                          "bytes_per_launch": gdn["in_bytes"] + ws_per_launch}}
     c = clocks.summary()
     line["clocks"] = c
