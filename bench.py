@@ -81,12 +81,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job rate under weak scaling: every rank processes units_per_rank
+    units, and the job takes as long as its slowest rank (ms_max)."""
+    return units_per_rank * world / (ms_max / 1e3)
 
 
 class ClockSampler:
@@ -377,7 +385,7 @@ def run_ours(args, world, rank, dev):
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
         gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
     hbm = peaks["hbm_gbs"]
-    value = pre["tokens"] * world / (pre["ms"] / 1e3)
+    value = job_throughput(pre["tokens"], pre["ms"], world)
 
     # Dominant prefill kernel and its roofline (HBM: the bytes it must move, i.e.
     # its inputs plus the per-chunk records it writes (prepare) or reads
@@ -443,7 +451,8 @@ def run_ours(args, world, rank, dev):
         g_ach = (gdn["in_bytes"] + ws_per_launch) / (gdn["prep_ms"] / 1e3) / 1e9
         line["gdn"] = {
             "workload": preset.name + "_gate_per_head",
-            "value": round(pre["tokens"] * world / (gdn["ms"] / 1e3), 1), "unit": "tokens/s",
+            "value": round(job_throughput(pre["tokens"], gdn["ms"], world), 1),
+            "unit": "tokens/s",
             "ms_per_step": round(gdn["ms"], 4),
             "kernels_ms": {"prepare": round(gdn["prep_ms"], 4), "carry": round(gdn["carry_ms"], 4)},
             "roofline": {"kernel": "prepare (one gate per head)", "bound": "hbm",
@@ -457,7 +466,7 @@ def run_ours(args, world, rank, dev):
         e = bench_e2e(pre, max(1, min(args.steps, args.e2e_steps)),
                       torch.cuda.current_stream())
         e_ms = max_over_ranks(e["ms"], world)
-        line["e2e"] = {"value": round(pre["tokens"] * world / (e_ms / 1e3), 1),
+        line["e2e"] = {"value": round(job_throughput(pre["tokens"], e_ms, world), 1),
                        "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
                        "d2h_bytes_per_step": e["d2h"], "ms_per_step": round(e_ms, 3)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
