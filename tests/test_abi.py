@@ -112,6 +112,37 @@ def test_decode_tokens_rejects(L, kw, status):
                                a["stream"]) == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(la=None), 1), (dict(B=0), 1), (dict(dk=96, dv=96), 2),
+    (dict(la=_fake(0x10004)), 3), (dict(ws_bytes=16), 4), (dict(algo=9), 1),
+    (dict(dt=0, algo=2), 2),
+])
+@pytest.mark.parametrize("fn", ["kda_gdn_chunk_fwd", "kda_gdn_chunk_fwd_prepare"])
+def test_gdn_chunk_fwd_rejects(L, fn, kw, status):
+    """The one-gate-per-head prefill checks its arguments like kda_chunk_fwd_ex."""
+    a = dict(q=_fake(), k=_fake(), v=_fake(), dt=1, la=_fake(), beta=_fake(), S0=None,
+             cu=None, n_seqs=0, B=1, T=64, H=2, dk=128, dv=128, scale=0.1, o=_fake(),
+             Sf=None, ws=_fake(), ws_bytes=1 << 40, algo=0, stream=None)
+    a.update(kw)
+    assert getattr(L, fn)(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["S0"],
+                          a["cu"], a["n_seqs"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                          a["scale"], a["o"], a["Sf"], a["ws"], a["ws_bytes"], a["algo"],
+                          a["stream"]) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=0), 1), (dict(la=None), 1), (dict(S=None), 1), (dict(dk=48, dv=48), 2),
+    (dict(S=_fake(0x10008)), 3), (dict(T=0, q=None, la=None), 0),
+])
+def test_gdn_decode_tokens_rejects(L, kw, status):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), dt=1, la=_fake(), beta=_fake(), S=_fake(),
+             N=4, T=3, H=2, dk=128, dv=128, scale=0.1, o=_fake(), stream=None)
+    a.update(kw)
+    assert L.kda_gdn_decode_tokens(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"],
+                                   a["S"], a["N"], a["T"], a["H"], a["dk"], a["dv"],
+                                   a["scale"], a["o"], a["stream"]) == status
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from gated_delta_rule_132_b200 import kda
     monkeypatch.setattr(kda, "_lib", None)
