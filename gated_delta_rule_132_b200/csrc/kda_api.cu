@@ -63,7 +63,7 @@ const char *kda_status_string(kda_status_t s)
     return "unknown status";
 }
 
-int kda_version(void) { return 100; }
+int kda_version(void) { return 200; }  // 0.2.0: multi-token decode and the GDN entry points
 
 size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
                                        kda_dtype_t dt, int algo)
