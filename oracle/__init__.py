@@ -3,6 +3,8 @@
 TEST INFRASTRUCTURE ONLY: imported by the test suite, the smoke check and the
 benchmark's CPU-baseline leg, never by the CUDA library.
 """
-from .kda_oracle import OracleLib, build, decode_step, default, forward, num_threads
+from .kda_oracle import (OracleLib, backward, build, decode_step, default, forward,
+                         num_threads)
 
-__all__ = ["OracleLib", "build", "decode_step", "default", "forward", "num_threads"]
+__all__ = ["OracleLib", "backward", "build", "decode_step", "default", "forward",
+           "num_threads"]

@@ -59,6 +59,11 @@ class OracleLib:
             _dp, _dp, _dp, _dp, _dp, _dp,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_double, _dp, ctypes.c_int]
+        lib.kda_oracle_backward.restype = ctypes.c_int
+        lib.kda_oracle_backward.argtypes = [
+            _dp, _dp, _dp, _dp, _dp, _dp, _i64p, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int]
         lib.kda_oracle_num_threads.restype = ctypes.c_int
         lib.kda_oracle_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -107,6 +112,49 @@ class OracleLib:
         if rc != 0:
             raise ValueError(f"kda_oracle_forward rejected its arguments (rc={rc})")
         return o, sf
+
+    def backward(self, q, k, v, log_alpha, beta, dO, S0=None, dS_final=None,
+                 cu_seqlens=None, scale=None, n_threads: int = 0):
+        """fp64 reverse-mode derivatives of L = <dO, o> + <dS_final, S_final>.
+
+        Inputs as :meth:`forward`, plus dO [B,T,H,dv] and dS_final [N,H,dk,dv] (or
+        None for zero). Returns a dict of float64 arrays with the inputs' shapes:
+        dq, dk, dv, dlog_alpha, dbeta and dS0 (the gradient of the initial state,
+        also when S0 is None, i.e. zero).
+        """
+        q, k, v, la, b, do = map(_f64, (q, k, v, log_alpha, beta, dO))
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        if k.shape != q.shape or la.shape != q.shape or v.shape[:3] != (B, T, H) \
+                or b.shape != (B, T, H) or do.shape != v.shape:
+            raise ValueError("shape mismatch")
+        if cu_seqlens is not None:
+            cu = np.ascontiguousarray(np.asarray(
+                cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                dtype=np.int64))
+            N = cu.shape[0] - 1
+            if B != 1:
+                raise ValueError("cu_seqlens needs B == 1")
+        else:
+            cu, N = None, B
+        s0, dsf = _f64(S0), _f64(dS_final)
+        for t, name in ((s0, "S0"), (dsf, "dS_final")):
+            if t is not None and t.shape != (N, H, dk, dv):
+                raise ValueError(f"{name} shape mismatch")
+        if scale is None:
+            scale = dk ** -0.5
+        out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
+               "dlog_alpha": np.zeros_like(la), "dbeta": np.zeros_like(b),
+               "dS0": np.zeros((N, H, dk, dv), dtype=np.float64)}
+        rc = self.lib.kda_oracle_backward(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0),
+            None if cu is None else cu.ctypes.data_as(_i64p), int(N),
+            int(B), int(T), int(H), int(dk), int(dv), float(scale), _ptr(do), _ptr(dsf),
+            _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_alpha"]),
+            _ptr(out["dbeta"]), _ptr(out["dS0"]), int(n_threads))
+        if rc != 0:
+            raise ValueError(f"kda_oracle_backward rejected its arguments (rc={rc})")
+        return out
 
     def decode_step(self, q, k, v, log_alpha, beta, S, scale=None, n_threads: int = 0):
         """One recurrent step for N sequences. q, k, log_alpha [N,H,dk]; v [N,H,dv];
@@ -166,3 +214,8 @@ def forward(*args, **kwargs):
 def decode_step(*args, **kwargs):
     """:meth:`OracleLib.decode_step` of the default build."""
     return default().decode_step(*args, **kwargs)
+
+
+def backward(*args, **kwargs):
+    """:meth:`OracleLib.backward` of the default build."""
+    return default().backward(*args, **kwargs)

@@ -357,3 +357,108 @@ def failing_pins(orc):
         if not ok:
             bad.append(name)
     return bad
+
+
+# ---------------------------------------------------------------------------
+# Backward pins. L = <dO, o> + <dS_final, S_final>; the oracle's backward must
+# give dL/d(every input). Checked against central differences of the (pinned)
+# forward and against a closed form where the rule makes one exact.
+BACKWARD_TOL = {
+    "b1_central_differences": 1e-7,
+    "b2_varlen_central_differences": 1e-7,
+    "b3_pure_decay_closed_form": 1e-12,
+}
+
+_GRAD_OF = (("q", "dq"), ("k", "dk"), ("v", "dv"), ("log_alpha", "dlog_alpha"),
+            ("beta", "dbeta"), ("S0", "dS0"))
+
+
+def _fd_gap(orc, x, dO, dSf, cu=None, h=1e-6):
+    """Largest gap between the backward and central differences of
+    L(x) = <dO, o> + <dSf, S_final>, over every element of every input,
+    relative to max(1, |finite difference|) per input."""
+    def loss(z):
+        o, sf = orc.forward(z["q"], z["k"], z["v"], z["log_alpha"], z["beta"], z["S0"], cu)
+        return float((o * dO).sum() + (sf * dSf).sum())
+
+    g = orc.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dO, x["S0"], dSf, cu)
+    worst = 0.0
+    for name, key in _GRAD_OF:
+        a = x[name]
+        fd = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            old = a[idx]
+            a[idx] = old + h
+            lp = loss(x)
+            a[idx] = old - h
+            lm = loss(x)
+            a[idx] = old
+            fd[idx] = (lp - lm) / (2 * h)
+        worst = max(worst, float(np.abs(fd - g[key]).max() / max(1.0, np.abs(fd).max())))
+    return worst
+
+
+def pin_b1_central_differences(orc):
+    """Every input's gradient against central differences, on a problem whose
+    sequences (70 tokens) cross the backward's 64-token replay blocks."""
+    q, k, v, la, b, S0 = _rand(101, B=2, T=70, H=1, dk=3, dv=2, unit_k=True)
+    r = np.random.default_rng(102)
+    S0 = S0 * 0.3
+    x = dict(q=q, k=k, v=v, log_alpha=la, beta=b, S0=S0)
+    return _fd_gap(orc, x, r.normal(size=v.shape), r.normal(size=S0.shape))
+
+
+def pin_b2_varlen_central_differences(orc):
+    """The same with packed sequences of 5, 0 and 7 tokens, one state each."""
+    q, k, v, la, b, _ = _rand(103, B=1, T=12, H=2, dk=3, dv=2, s0=False, unit_k=True)
+    r = np.random.default_rng(104)
+    S0 = r.normal(size=(3, 2, 3, 2)) * 0.3
+    x = dict(q=q, k=k, v=v, log_alpha=la, beta=b, S0=S0)
+    cu = np.array([0, 5, 5, 12], dtype=np.int64)
+    return _fd_gap(orc, x, r.normal(size=v.shape), r.normal(size=S0.shape), cu)
+
+
+def pin_b3_pure_decay_closed_form(orc):
+    """beta = 0 leaves only the decay: S_t = Diag(e^{g_t}) S0 with g_t the
+    cumulative log_alpha, so o_t = scale S0^T Diag(e^{g_t}) q_t and
+        dq_t   = scale Diag(e^{g_t}) S0 dO_t,
+        dS0    = sum_t scale Diag(e^{g_t}) q_t dO_t^T + Diag(e^{g_T}) dS_final,
+        dlog_alpha_s[i] = sum_{t>=s} scale q_t[i] e^{g_t[i]} (S0 dO_t)_i
+                          + e^{g_T[i]} sum_j S0_ij dS_final_ij,
+        dk = dv = 0."""
+    q, k, v, la, _, S0 = _rand(105, B=1, T=9, H=1, dk=4, dv=3)
+    b = np.zeros((1, 9, 1))
+    r = np.random.default_rng(106)
+    dO, dSf = r.normal(size=v.shape), r.normal(size=S0.shape)
+    scale = 0.5
+    g = orc.backward(q, k, v, la, b, dO, S0, dSf, scale=scale)
+    G = np.cumsum(la[0, :, 0], axis=0)  # [T, dk]
+    s0 = S0[0, 0]
+    dq = np.stack([scale * np.exp(G[t]) * (s0 @ dO[0, t, 0]) for t in range(9)])
+    dS0 = sum(scale * np.outer(np.exp(G[t]) * q[0, t, 0], dO[0, t, 0]) for t in range(9))
+    dS0 = dS0 + np.exp(G[-1])[:, None] * dSf[0, 0]
+    per_t = np.stack([scale * q[0, t, 0] * np.exp(G[t]) * (s0 @ dO[0, t, 0]) for t in range(9)])
+    dla = np.cumsum(per_t[::-1], axis=0)[::-1] + np.exp(G[-1]) * (s0 * dSf[0, 0]).sum(axis=1)
+    return _maxdiff((g["dq"][0, :, 0], dq), (g["dS0"][0, 0], dS0),
+                    (g["dlog_alpha"][0, :, 0], dla), (g["dk"], 0 * k), (g["dv"], 0 * v))
+
+
+BACKWARD_ALL = {
+    "b1_central_differences": pin_b1_central_differences,
+    "b2_varlen_central_differences": pin_b2_varlen_central_differences,
+    "b3_pure_decay_closed_form": pin_b3_pure_decay_closed_form,
+}
+
+
+def failing_backward_pins(orc):
+    """Names of the backward pins that ``orc`` violates (an exception counts)."""
+    bad = []
+    for name, fn in BACKWARD_ALL.items():
+        try:
+            e = fn(orc)
+            ok = np.isfinite(e) and e <= BACKWARD_TOL[name]
+        except Exception:  # noqa: BLE001 - a crash or rejection is a failure
+            ok = False
+        if not ok:
+            bad.append(name)
+    return bad
