@@ -11,7 +11,7 @@ import importlib
 from . import inputs  # noqa: F401  (no CUDA needed)
 
 _EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_prepare", "kda_chunk_fwd_carry",
-            "kda_decode_step", "kda_decode_tokens", "kda_gdn_chunk_fwd",
+            "kda_decode_step", "kda_decode_tokens", "kda_gdn_chunk_fwd", "kda_chunk_bwd",
             "kda_chunk_fwd_workspace_size",
             "ChunkFwdCall", "lib", "KdaError")
 

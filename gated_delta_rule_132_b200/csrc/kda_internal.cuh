@@ -79,6 +79,11 @@ cudaError_t launch_simt_prefill(const Problem &p, void *workspace, int phases,
 cudaError_t launch_tc_prefill(const Problem &p, void *workspace, int phases,
                               cudaStream_t stream);
 bool tc_supported(const Problem &p);
+// Backward of the prefill (fp32 CUDA cores): gradients of <dO, o> + <dS_final, S_final>.
+WorkspaceLayout bwd_workspace_layout(const Problem &p);
+cudaError_t launch_backward(const Problem &p, const void *dO, const float *dS_final,
+                            float *gq, float *gk, float *gv, float *gla, float *gbeta,
+                            float *gS0, void *workspace, cudaStream_t stream);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -66,6 +66,12 @@ def lib() -> ctypes.CDLL:
         L.kda_decode_step.restype = _i
         L.kda_decode_step.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                                       _vp, _vp]
+        L.kda_chunk_bwd_workspace_size.restype = _sz
+        L.kda_chunk_bwd_workspace_size.argtypes = [_i] * 7
+        for fn in ("kda_chunk_bwd", "kda_gdn_chunk_bwd"):
+            getattr(L, fn).restype = _i
+            getattr(L, fn).argtypes = ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                        _i, _i, _f] + [_vp] * 9 + [_sz, _vp])
         for fn in ("kda_decode_tokens", "kda_gdn_decode_tokens"):
             getattr(L, fn).restype = _i
             getattr(L, fn).argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -216,6 +222,58 @@ def kda_gdn_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=
     """
     return ChunkFwdCall(q, k, v, log_alpha, beta, S0, cu_seqlens, scale, output_final_state,
                         workspace, o, S_final, algo, gate="head").run(stream)
+
+
+def kda_chunk_bwd(q, k, v, log_alpha, beta, dO, S0=None, cu_seqlens=None, scale=None,
+                  dS_final=None, want_dS0=True, workspace=None, gate="channel", stream=None):
+    """Backward of the prefill (C: ``kda_chunk_bwd`` / ``kda_gdn_chunk_bwd``): the
+    gradients of <dO, o> + <dS_final, S_final>.
+
+    Arguments as :func:`kda_chunk_fwd` (``gate="head"``: log_alpha [B,T,H]), plus
+    dO [B,T,H,dv] in q's dtype and dS_final [N,H,dk,dv] fp32 or None. Returns a dict
+    of fp32 tensors dq, dk, dv, dlog_alpha, dbeta and dS0 (None unless want_dS0).
+    """
+    if gate not in ("channel", "head"):
+        raise ValueError(f"gate must be 'channel' or 'head', not {gate!r}")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dtype = q.dtype
+    _dt(q)
+    for t, name in ((q, "q"), (k, "k")):
+        _need(t, name, dtype, (B, T, H, dk))
+    _need(v, "v", dtype, (B, T, H, dv))
+    _need(dO, "dO", dtype, (B, T, H, dv))
+    la_shape = (B, T, H, dk) if gate == "channel" else (B, T, H)
+    _need(log_alpha, "log_alpha", torch.float32, la_shape)
+    _need(beta, "beta", torch.float32, (B, T, H))
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.shape[0] - 1
+    else:
+        N = B
+    for t, name in ((S0, "S0"), (dS_final, "dS_final")):
+        if t is not None:
+            _need(t, name, torch.float32, (N, H, dk, dv))
+    if scale is None:
+        scale = dk ** -0.5
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty((B, T, H, dk), **f32), "dk": torch.empty((B, T, H, dk), **f32),
+         "dv": torch.empty((B, T, H, dv), **f32), "dlog_alpha": torch.empty(la_shape, **f32),
+         "dbeta": torch.empty((B, T, H), **f32),
+         "dS0": torch.empty((N, H, dk, dv), **f32) if want_dS0 else None}
+    n_seqs = N if cu_seqlens is not None else 0
+    need = int(lib().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, n_seqs, _dt(q)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    fn = "kda_chunk_bwd" if gate == "channel" else "kda_gdn_chunk_bwd"
+    st = getattr(lib(), fn)(
+        _p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S0), _p(cu_seqlens),
+        int(n_seqs), B, T, H, dk, dv, float(scale), _p(dO), _p(dS_final), _p(g["dq"]),
+        _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]), _p(g["dbeta"]), _p(g["dS0"]),
+        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != 0:
+        raise KdaError(fn, st)
+    return g
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, S, scale=None, o=None, stream=None):

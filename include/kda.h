@@ -228,6 +228,43 @@ kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v,
                                    int dv, float scale, void *o, void *stream);
 
 /*
+ * Backward of the prefill (for training; the pages state only the forward rule,
+ * so this is the rule's derivative, taken token by token in reverse order):
+ * the gradients of
+ *     L = <dO, o> + <dS_final, S_final>
+ * with respect to q, k, v, log_alpha, beta and S0, for the arguments of
+ * kda_chunk_fwd (same layouts, sequences and scale). Computed in fp32 on CUDA
+ * cores for every supported head size; the states are replayed from
+ * checkpoints kept every 64 tokens in the workspace.
+ *   dO              qkv_dtype [B, T, H, dv]
+ *   dS_final        fp32 [N, H, dk, dv] or NULL (zero)
+ *   grad_q, grad_k  fp32 [B, T, H, dk]       grad_v     fp32 [B, T, H, dv]
+ *   grad_log_alpha  fp32 [B, T, H, dk]       grad_beta  fp32 [B, T, H]
+ *   grad_S0         fp32 [N, H, dk, dv] or NULL (not returned)
+ * Workspace: kda_chunk_bwd_workspace_size bytes. Errors as kda_chunk_fwd_ex.
+ * Tokens outside every sequence (cu_seqlens ending before B*T) are not written.
+ * kda_gdn_chunk_bwd: the same for one gate per token and head (log_alpha and
+ * grad_log_alpha fp32 [B, T, H]).
+ */
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                    kda_dtype_t qkv_dtype);
+kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                           const float *log_alpha, const float *beta, const float *S0,
+                           const int32_t *cu_seqlens, int n_seqs, int B, int T, int H, int dk,
+                           int dv, float scale, const void *dO, const float *dS_final,
+                           float *grad_q, float *grad_k, float *grad_v, float *grad_log_alpha,
+                           float *grad_beta, float *grad_S0, void *workspace,
+                           size_t workspace_bytes, void *stream);
+kda_status_t kda_gdn_chunk_bwd(const void *q, const void *k, const void *v,
+                               kda_dtype_t qkv_dtype, const float *log_alpha,
+                               const float *beta, const float *S0, const int32_t *cu_seqlens,
+                               int n_seqs, int B, int T, int H, int dk, int dv, float scale,
+                               const void *dO, const float *dS_final, float *grad_q,
+                               float *grad_k, float *grad_v, float *grad_log_alpha,
+                               float *grad_beta, float *grad_S0, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
  * kda_chunk_fwd_noalloc — the chunked prefill for callers that cannot allocate
  * device memory (no counterpart in the paper; it exists for callers such as a
  * plugin whose host application owns all device memory, or code that must not

@@ -143,6 +143,33 @@ def test_gdn_decode_tokens_rejects(L, kw, status):
                                    a["scale"], a["o"], a["stream"]) == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(dO=None), 1), (dict(gq=None), 1), (dict(gbeta=None), 1),
+    (dict(B=0), 1), (dict(dk=96, dv=96), 2), (dict(dt=5), 2), (dict(gla=_fake(0x10004)), 3),
+    (dict(dO=_fake(0x10002)), 3), (dict(ws=None), 4), (dict(ws_bytes=64), 4),
+    (dict(scale=float("nan")), 1),
+])
+@pytest.mark.parametrize("fn", ["kda_chunk_bwd", "kda_gdn_chunk_bwd"])
+def test_chunk_bwd_rejects(L, fn, kw, status):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), dt=1, la=_fake(), beta=_fake(), S0=None,
+             cu=None, n_seqs=0, B=1, T=64, H=2, dk=128, dv=128, scale=0.1, dO=_fake(),
+             dSf=None, gq=_fake(), gk=_fake(), gv=_fake(), gla=_fake(), gbeta=_fake(),
+             gS0=None, ws=_fake(), ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    assert getattr(L, fn)(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["S0"],
+                          a["cu"], a["n_seqs"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                          a["scale"], a["dO"], a["dSf"], a["gq"], a["gk"], a["gv"],
+                          a["gla"], a["gbeta"], a["gS0"], a["ws"], a["ws_bytes"],
+                          a["stream"]) == status
+
+
+def test_chunk_bwd_workspace_size(L):
+    a = L.kda_chunk_bwd_workspace_size(1, 4096, 8, 128, 128, 0, 1)
+    b = L.kda_chunk_bwd_workspace_size(1, 4097, 8, 128, 128, 0, 1)
+    assert 0 < a < b
+    assert L.kda_chunk_bwd_workspace_size(1, 100, 4, 96, 96, 0, 0) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from gated_delta_rule_132_b200 import kda
     monkeypatch.setattr(kda, "_lib", None)

@@ -1,0 +1,70 @@
+"""kda_chunk_bwd / kda_gdn_chunk_bwd on the GPU against the fp64 oracle's
+backward (itself pinned by central differences of the forward): every gradient
+of <dO, o> + <dS_final, S_final>, element by element, on the same inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from common import rel_l2
+from gated_delta_rule_132_b200 import inputs as I
+from gated_delta_rule_132_b200 import kda
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-4  # fp32 arithmetic on both gate forms; the oracle sees the same input values
+KEYS = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0")
+
+
+def _problem(B, T, H, d, dtype, seed, lengths=None, s0=True):
+    x = I.make_prefill(B, T, H, d, dtype, gate_shift=-1.0, s0_std=0.1 if s0 else 0.0,
+                       seed=seed, lengths=lengths)
+    g = torch.Generator().manual_seed(seed + 1)
+    N = B if lengths is None else len(lengths)
+    dO = torch.randn(x["v"].shape, generator=g).to(dtype)
+    dSf = torch.randn((N, H, d, d), generator=g) if s0 else None
+    return x, dO, dSf
+
+
+def _check(x, dO, dSf, gate="channel"):
+    la = x["log_alpha"] if gate == "channel" else x["log_alpha"][..., 0].contiguous()
+    la_full = la if gate == "channel" else la[..., None].expand_as(x["log_alpha"]).contiguous()
+    dev = lambda t: None if t is None else t.cuda()
+    got = kda.kda_chunk_bwd(dev(x["q"]), dev(x["k"]), dev(x["v"]), la.cuda(), dev(x["beta"]),
+                            dO.cuda(), dev(x["S0"]), dev(x["cu_seqlens"]), x["scale"],
+                            dev(dSf), gate=gate)
+    torch.cuda.synchronize()
+    ref = oracle.backward(x["q"], x["k"], x["v"], la_full, x["beta"], dO, x["S0"], dSf,
+                          x["cu_seqlens"], scale=x["scale"])
+    if gate == "head":
+        ref["dlog_alpha"] = ref["dlog_alpha"].sum(axis=-1)
+    errs = {key: rel_l2(got[key], ref[key]) for key in KEYS}
+    assert all(np.isfinite(e) and e <= TOL for e in errs.values()), errs
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 32), (torch.float32, 64),
+                                     (torch.float32, 128), (torch.bfloat16, 128)])
+def test_backward_crossing_checkpoints(dtype, d):
+    """70 tokens per sequence: the replay crosses a 64-token checkpoint."""
+    _check(*_problem(2, 70, 2, d, dtype, seed=700 + d))
+
+
+def test_backward_varlen_with_empty_sequence():
+    _check(*_problem(1, 0, 2, 64, torch.float32, seed=710, lengths=[5, 0, 65, 130]))
+
+
+@pytest.mark.parametrize("gate_dtype", [torch.float32, torch.bfloat16])
+def test_backward_one_gate_per_head(gate_dtype):
+    _check(*_problem(2, 100, 2, 128 if gate_dtype == torch.bfloat16 else 32, gate_dtype,
+                     seed=720), gate="head")
+
+
+def test_backward_without_states():
+    """S0 and dS_final absent (zero); the initial-state gradient still comes back."""
+    x, dO, dSf = _problem(1, 90, 3, 64, torch.float32, seed=730, s0=False)
+    _check(x, dO, dSf)
+
+
+def test_backward_long_bf16():
+    """300 tokens (five checkpoint blocks), 4 heads, d = 128, bf16 inputs."""
+    _check(*_problem(1, 300, 4, 128, torch.bfloat16, seed=740))
