@@ -250,6 +250,45 @@ def bench_gdn(pre, steps, warmup, world):
                 carry_ms=statistics.mean(p[1] for p in per), in_bytes=in_b)
 
 
+# The backward (kda_chunk_bwd) on the long workload's shape cut to its first 8192
+# tokens: fp32 CUDA-core arithmetic, ~28 dk*dv flop per token and head (two
+# forward replays and the reverse step).
+BWD_T = 8192
+BWD_FLOP_PER_TOKEN_HEAD = 28 * 128 * 128
+# fp32 FMA peak from the SM count, FP32 lanes per SM and the maximum SM clock:
+# 148 x 128 x 2 flop x 1.965 GHz.
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bench_backward(steps, warmup, world, rank, dev):
+    from gated_delta_rule_132_b200 import kda
+    P = I.LONG
+    devs = f"cuda:{dev}"
+    x = I.make_prefill(1, BWD_T, P.H, P.d, P.dtype, P.gate_shift, 0.0, P.seed + 1000 * rank,
+                       device=devs)
+    g = torch.Generator(device=devs).manual_seed(P.seed + 7 + 1000 * rank)
+    dO = torch.randn(x["v"].shape, generator=g, device=devs).to(P.dtype)
+    ws = torch.empty(int(kda.lib().kda_chunk_bwd_workspace_size(1, BWD_T, P.H, P.d, P.d, 0, 1)),
+                     dtype=torch.uint8, device=devs)
+    args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dO)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        kda.kda_chunk_bwd(*args, workspace=ws)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    def step(i, ev):
+        ev[0].record(stream)
+        kda.kda_chunk_bwd(*args, workspace=ws)
+        ev[1].record(stream)
+
+    total_ms, per = time_region(step, steps, stream, marks=2)
+    barrier(world)
+    return dict(ms=max_over_ranks(total_ms / steps, world),
+                kern_ms=statistics.mean(p[0] for p in per), tokens=BWD_T,
+                token_heads=BWD_T * P.H, workload=f"long_bf16_B1_H{P.H}_T{BWD_T}_d{P.d}")
+
+
 def bench_decode(P, steps, warmup, world, rank, dev):
     from gated_delta_rule_132_b200 import kda
     devs = f"cuda:{dev}"
@@ -384,6 +423,8 @@ def run_ours(args, world, rank, dev):
         dtok = None if args.no_decode else bench_decode_tokens(
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
         gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
+        bwd = None if args.no_backward else bench_backward(
+            min(args.steps, 3), args.warmup, world, rank, dev)
     hbm = peaks["hbm_gbs"]
     value = job_throughput(pre["tokens"], pre["ms"], world)
 
@@ -460,6 +501,18 @@ def run_ours(args, world, rank, dev):
                          "frac": round(g_ach / hbm, 4),
                          "traffic": TRAFFIC_PER_RECORD["gdn_prepare"] * pre["records"],
                          "bytes_per_launch": gdn["in_bytes"] + ws_per_launch}}
+    if bwd is not None:
+        tf = bwd["token_heads"] * BWD_FLOP_PER_TOKEN_HEAD / (bwd["kern_ms"] / 1e3) / 1e12
+        line["backward"] = {
+            "workload": bwd["workload"] + "_backward",
+            "value": round(job_throughput(bwd["tokens"], bwd["ms"], world), 1),
+            "unit": "tokens/s", "ms_per_step": round(bwd["ms"], 3),
+            "steps": min(args.steps, 3), "warmup": args.warmup,
+            "roofline": {"kernel": "backward (fp32 CUDA cores)", "bound": "alu",
+                         "achieved": round(tf, 3), "peak": round(FP32_PEAK_TFLOPS, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / FP32_PEAK_TFLOPS, 4),
+                         "traffic": None, "peak_source": "derived: 148 SMs x 128 fp32 lanes "
+                                                         "x 2 flop x 1.965 GHz"}}
     c = clocks.summary()
     line["clocks"] = c
     if not args.no_e2e:
@@ -525,6 +578,8 @@ def main():
     ap.add_argument("--workload", choices=["long", "chunked", "varlen"], default="long",
                     help="prefill workload (default: the long-context one)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward (kda_chunk_bwd) measurement")
     ap.add_argument("--no-gdn", action="store_true",
                     help="skip the one-gate-per-head (GDN) variant of the prefill")
     ap.add_argument("--e2e-steps", type=int, default=3)

@@ -17,14 +17,16 @@
 // and dS0 = G once the first token is undone.
 //
 // One CTA per (sequence, head) with D threads (D = dk = dv): thread i owns row
-// i of the state or gradient in the row phases and column i in the column
-// phases; both matrices sit in shared memory with rows padded to D + 1 floats,
-// so row and column sweeps are free of bank conflicts. The states the backward
+// i of a matrix in the row phases and column i in the column phases; the two
+// state buffers and G sit in shared memory with rows padded to D + 1 floats, so
+// row and column sweeps are free of bank conflicts. The states the backward
 // needs come from a replay of the forward: a first pass stores the state at
 // every 64-token chunk start (per (chunk, head), like the prefill's records);
 // each chunk, last to first, is then replayed from its checkpoint into a
-// per-(sequence, head) buffer of its 65 states and walked backwards.
-// Every step is a plain fp32 loop; this is the correctness-first backward.
+// per-(sequence, head) buffer of its 65 states and walked backwards. The walk
+// keeps S_t in one buffer and fetches S_{t-1} into the other (float4 loads
+// issued before the read-out sweep), applying Diag(alpha) on the fly, so
+// S_{t-1} is the next step's S_t unchanged. Plain fp32 loops throughout.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -54,13 +56,39 @@ __device__ __forceinline__ float ld(const void *p, size_t i)
 template <int D>
 __device__ __forceinline__ void store_mat(float *dst, const float *sm)
 {
-    for (int e = threadIdx.x; e < D * D; e += D) dst[e] = sm[(e / D) * (D + 1) + e % D];
+#pragma unroll 4
+    for (int e4 = threadIdx.x; e4 < D * D / 4; e4 += D) {
+        const int r = (4 * e4) / D, c = (4 * e4) % D;
+        const float *x = sm + r * (D + 1) + c;
+        reinterpret_cast<float4 *>(dst)[e4] = make_float4(x[0], x[1], x[2], x[3]);
+    }
+}
+
+// Global -> registers (D / 4 float4 per thread, all in flight), then -> shared.
+template <int D>
+__device__ __forceinline__ void fetch_mat(float4 *reg, const float *src)
+{
+#pragma unroll
+    for (int m = 0; m < D / 4; ++m) reg[m] = reinterpret_cast<const float4 *>(src)[threadIdx.x + D * m];
+}
+
+template <int D>
+__device__ __forceinline__ void put_mat(float *sm, const float4 *reg)
+{
+#pragma unroll
+    for (int m = 0; m < D / 4; ++m) {
+        const int e = 4 * (threadIdx.x + D * m), r = e / D, c = e % D;
+        float *x = sm + r * (D + 1) + c;
+        x[0] = reg[m].x; x[1] = reg[m].y; x[2] = reg[m].z; x[3] = reg[m].w;
+    }
 }
 
 template <int D>
 __device__ __forceinline__ void load_mat(float *sm, const float *src)
 {
-    for (int e = threadIdx.x; e < D * D; e += D) sm[(e / D) * (D + 1) + e % D] = src[e];
+    float4 reg[D / 4];
+    fetch_mat<D>(reg, src);
+    put_mat<D>(sm, reg);
 }
 
 template <int D, typename TIn>
@@ -68,8 +96,9 @@ __global__ void __launch_bounds__(D) bwd_kernel(BwdParams p)
 {
     extern __shared__ float smem[];
     constexpr int P1 = D + 1;
-    float *S = smem;             // [D][D+1]: state (forward, replay) / P, Q (backward)
-    float *G = S + D * P1;       // [D][D+1]: dL/dS
+    float *S = smem;             // [D][D+1]: state (forward, replay); S_t or S_{t-1} (backward)
+    float *S2 = S + D * P1;      // [D][D+1]: the other of S_t, S_{t-1} (backward)
+    float *G = S2 + D * P1;      // [D][D+1]: dL/dS
     float *sk = G + D * P1;      // token vectors
     float *sq = sk + D;
     float *sa = sq + D;          // alpha
@@ -138,32 +167,30 @@ __global__ void __launch_bounds__(D) bwd_kernel(BwdParams p)
             store_mat<D>(blk + (size_t)(t - a + 1) * D * D, S);
         }
         __syncthreads();
+        // S holds S_e, the state after the block: S_t for t = e - 1
+        float *cur = S, *prev = S2;
         for (int t = e - 1; t >= a; --t) {
             const size_t th = (size_t)t * H + h;
             load_token(t);
             const float bt = sred[32];
-            // read-out: S <- Q = S_t
-            load_mat<D>(S, blk + (size_t)(t - a + 1) * D * D);
-            __syncthreads();
+            float4 reg[D / 4];
+            fetch_mat<D>(reg, blk + (size_t)(t - a) * D * D);  // S_{t-1}, in flight
+            // read-out with S_t
             {
                 float acc = 0.f;
                 for (int j = 0; j < D; ++j) {
                     G[i * P1 + j] += p.scale * sq[i] * sdo[j];
-                    acc += S[i * P1 + j] * sdo[j];
+                    acc += cur[i * P1 + j] * sdo[j];
                 }
                 p.gq[th * D + i] = p.scale * acc;
             }
+            put_mat<D>(prev, reg);
             __syncthreads();
-            // S <- S' = Diag(alpha) S_{t-1}
-            load_mat<D>(S, blk + (size_t)(t - a) * D * D);
-            __syncthreads();
-            for (int j = 0; j < D; ++j) S[i * P1 + j] *= sa[i];
-            __syncthreads();
-            // column i: w_i, g_i, dv_i and this column's share of dbeta
+            // column i: w_i, g_i, dv_i and this column's share of dbeta (S' = Diag(alpha) S_{t-1})
             {
                 float ks = 0.f, gk = 0.f;
                 for (int r = 0; r < D; ++r) {
-                    ks += S[r * P1 + i] * sk[r];
+                    ks += sa[r] * prev[r * P1 + i] * sk[r];
                     gk += G[r * P1 + i] * sk[r];
                 }
                 const float w = sv[i] - ks;
@@ -183,41 +210,44 @@ __global__ void __launch_bounds__(D) bwd_kernel(BwdParams p)
             }
             // row i: dk_i, dS' row, dlog_alpha_i, then G <- Diag(alpha) dS'
             {
-                float gw = 0.f, sgv = 0.f;
+                const float al = sa[i];
+                float gw = 0.f, pg = 0.f;
                 for (int j = 0; j < D; ++j) {
                     gw += G[i * P1 + j] * sw[j];
-                    sgv += S[i * P1 + j] * sg[j];
+                    pg += prev[i * P1 + j] * sg[j];
                 }
-                p.gk[th * D + i] = bt * (gw - sgv);
+                p.gk[th * D + i] = bt * (gw - al * pg);
                 float dl = 0.f;
                 for (int j = 0; j < D; ++j) {
                     const float d = G[i * P1 + j] - bt * sk[i] * sg[j];
-                    dl += d * S[i * P1 + j];
-                    G[i * P1 + j] = sa[i] * d;
+                    dl += d * prev[i * P1 + j];
+                    G[i * P1 + j] = al * d;
                 }
+                dl *= al;
                 if (p.gate_per_channel) p.gla[th * D + i] = dl;
                 else {
                     // one gate per head: its gradient is the sum over the channels
-                    float s = dl;
+                    float s2 = dl;
 #pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-                    if ((i & 31) == 0) sred2[i >> 5] = s;
+                    for (int off = 16; off > 0; off >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+                    if ((i & 31) == 0) sred2[i >> 5] = s2;
                 }
             }
             __syncthreads();
             if (!p.gate_per_channel && i == 0) {
-                float s = 0.f;
-                for (int q = 0; q < D / 32; ++q) s += sred2[q];
-                p.gla[th] = s;
+                float s2 = 0.f;
+                for (int q = 0; q < D / 32; ++q) s2 += sred2[q];
+                p.gla[th] = s2;
             }
             __syncthreads();
+            float *tmp = cur; cur = prev; prev = tmp;  // S_{t-1} is the next step's S_t
         }
     }
     if (p.gS0)
         for (int j = 0; j < D; ++j) p.gS0[((size_t)unit * D + i) * D + j] = G[i * P1 + j];
 }
 
-template <int D> constexpr size_t bwd_smem() { return sizeof(float) * (2 * D * (D + 1) + 7 * D + 65); }
+template <int D> constexpr size_t bwd_smem() { return sizeof(float) * (3 * D * (D + 1) + 7 * D + 65); }
 
 template <int D, typename TIn>
 cudaError_t launch_d(const BwdParams &p, cudaStream_t st)
