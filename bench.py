@@ -260,15 +260,15 @@ BWD_FLOP_PER_TOKEN_HEAD = 28 * 128 * 128
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def bench_backward(steps, warmup, world, rank, dev):
+def bench_backward(steps, warmup, world, rank, dev, T_b=BWD_T):
     from gated_delta_rule_132_b200 import kda
     P = I.LONG
     devs = f"cuda:{dev}"
-    x = I.make_prefill(1, BWD_T, P.H, P.d, P.dtype, P.gate_shift, 0.0, P.seed + 1000 * rank,
+    x = I.make_prefill(1, T_b, P.H, P.d, P.dtype, P.gate_shift, 0.0, P.seed + 1000 * rank,
                        device=devs)
     g = torch.Generator(device=devs).manual_seed(P.seed + 7 + 1000 * rank)
     dO = torch.randn(x["v"].shape, generator=g, device=devs).to(P.dtype)
-    ws = torch.empty(int(kda.lib().kda_chunk_bwd_workspace_size(1, BWD_T, P.H, P.d, P.d, 0, 1)),
+    ws = torch.empty(int(kda.lib().kda_chunk_bwd_workspace_size(1, T_b, P.H, P.d, P.d, 0, 1)),
                      dtype=torch.uint8, device=devs)
     args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dO)
     stream = torch.cuda.current_stream()
@@ -285,8 +285,8 @@ def bench_backward(steps, warmup, world, rank, dev):
     total_ms, per = time_region(step, steps, stream, marks=2)
     barrier(world)
     return dict(ms=max_over_ranks(total_ms / steps, world),
-                kern_ms=statistics.mean(p[0] for p in per), tokens=BWD_T,
-                token_heads=BWD_T * P.H, workload=f"long_bf16_B1_H{P.H}_T{BWD_T}_d{P.d}")
+                kern_ms=statistics.mean(p[0] for p in per), tokens=T_b,
+                token_heads=T_b * P.H, workload=f"long_bf16_B1_H{P.H}_T{T_b}_d{P.d}")
 
 
 def bench_decode(P, steps, warmup, world, rank, dev):
@@ -424,7 +424,7 @@ def run_ours(args, world, rank, dev):
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
         gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
         bwd = None if args.no_backward else bench_backward(
-            min(args.steps, 3), args.warmup, world, rank, dev)
+            min(args.steps, 3), args.warmup, world, rank, dev, args.bwd_tokens)
     hbm = peaks["hbm_gbs"]
     value = job_throughput(pre["tokens"], pre["ms"], world)
 
@@ -580,6 +580,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward (kda_chunk_bwd) measurement")
+    ap.add_argument("--bwd-tokens", type=int, default=BWD_T,
+                    help="tokens of the backward measurement (all 32 heads)")
     ap.add_argument("--no-gdn", action="store_true",
                     help="skip the one-gate-per-head (GDN) variant of the prefill")
     ap.add_argument("--e2e-steps", type=int, default=3)
