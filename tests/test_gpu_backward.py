@@ -45,7 +45,7 @@ def _check(x, dO, dSf, gate="channel"):
 @pytest.mark.parametrize("dtype,d", [(torch.float32, 32), (torch.float32, 64),
                                      (torch.float32, 128), (torch.bfloat16, 128)])
 def test_backward_crossing_checkpoints(dtype, d):
-    """70 tokens per sequence: the replay crosses a 64-token checkpoint."""
+    """70 tokens per sequence: two full 32-token replay blocks and a ragged one."""
     _check(*_problem(2, 70, 2, d, dtype, seed=700 + d))
 
 
@@ -68,3 +68,40 @@ def test_backward_without_states():
 def test_backward_long_bf16():
     """300 tokens (five checkpoint blocks), 4 heads, d = 128, bf16 inputs."""
     _check(*_problem(1, 300, 4, 128, torch.bfloat16, seed=740))
+
+
+def test_backward_block_edges():
+    """Lengths around the 32-token replay block and the 64-token chunk."""
+    _check(*_problem(1, 0, 2, 64, torch.float32, seed=750, lengths=[1, 31, 32, 33, 64, 65]))
+
+
+def test_backward_leaves_tokens_outside_sequences_unwritten():
+    """cu_seqlens ending before B*T: the trailing tokens keep what the caller put there;
+    the covered ones match the oracle (they do not depend on later sequences)."""
+    x, dO, dSf = _problem(1, 0, 2, 128, torch.float32, seed=760, lengths=[40, 30, 10])
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dO, x["S0"], dSf,
+                          x["cu_seqlens"], scale=x["scale"])
+    cu = x["cu_seqlens"][:3].cuda()
+    B, T, H, d = x["q"].shape
+    sentinel = 12345.0
+    out = {key: torch.full(ref[key].shape, sentinel, device="cuda") for key in KEYS}
+    out["dS0"] = torch.full((2, H, d, d), sentinel, device="cuda")
+    dev = {key: x[key].cuda() for key in ("q", "k", "v", "log_alpha", "beta", "S0")}
+    dS0_in = dev["S0"][:2].contiguous()
+    dSf2 = dSf[:2].contiguous().cuda()
+    dOc = dO.cuda()
+    need = int(kda.lib().kda_chunk_bwd_workspace_size(B, T, H, d, d, 2, kda._dt(dev["q"])))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    st = kda.lib().kda_chunk_bwd(
+        kda._p(dev["q"]), kda._p(dev["k"]), kda._p(dev["v"]), kda._dt(dev["q"]),
+        kda._p(dev["log_alpha"]), kda._p(dev["beta"]), kda._p(dS0_in), kda._p(cu), 2, B, T, H,
+        d, d, float(x["scale"]), kda._p(dOc), kda._p(dSf2), kda._p(out["dq"]),
+        kda._p(out["dk"]), kda._p(out["dv"]), kda._p(out["dlog_alpha"]), kda._p(out["dbeta"]),
+        kda._p(out["dS0"]), kda._p(ws), need, kda._stream(None))
+    assert st == 0
+    torch.cuda.synchronize()
+    for key in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        got = out[key].cpu()
+        assert torch.all(got[:, 70:] == sentinel), key
+        assert rel_l2(got[:, :70], ref[key][:, :70]) <= TOL, key
+    assert rel_l2(out["dS0"].cpu(), ref["dS0"][:2]) <= TOL
