@@ -255,6 +255,10 @@ def bench_gdn(pre, steps, warmup, world):
 # forward replays and the reverse step).
 BWD_T = 8192
 BWD_FLOP_PER_TOKEN_HEAD = 28 * 128 * 128
+# DRAM bytes (read + write) of bwd_kernel per token and head: one ncu capture at
+# T = 1024 (163.7 MB read + 1573.9 MB written), scaled by token-heads. Most of it
+# is the per-block replay buffer written back from L2.
+BWD_TRAFFIC_PER_TOKEN_HEAD = 53_027
 # fp32 FMA peak from the SM count, FP32 lanes per SM and the maximum SM clock:
 # 148 x 128 x 2 flop x 1.965 GHz.
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -511,8 +515,9 @@ def run_ours(args, world, rank, dev):
             "roofline": {"kernel": "backward (fp32 CUDA cores)", "bound": "alu",
                          "achieved": round(tf, 3), "peak": round(FP32_PEAK_TFLOPS, 1),
                          "unit": "TFLOP/s", "frac": round(tf / FP32_PEAK_TFLOPS, 4),
-                         "traffic": None, "peak_source": "derived: 148 SMs x 128 fp32 lanes "
-                                                         "x 2 flop x 1.965 GHz"}}
+                         "traffic": BWD_TRAFFIC_PER_TOKEN_HEAD * bwd["token_heads"],
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz",
+                         "timed": "whole kda_chunk_bwd call (plan, bwd_kernel, reduction)"}}
     c = clocks.summary()
     line["clocks"] = c
     if not args.no_e2e:

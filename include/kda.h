@@ -235,7 +235,9 @@ kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v,
  * with respect to q, k, v, log_alpha, beta and S0, for the arguments of
  * kda_chunk_fwd (same layouts, sequences and scale). Computed in fp32 on CUDA
  * cores for every supported head size; the states are replayed from
- * checkpoints kept every 64 tokens in the workspace.
+ * checkpoints kept every 32 tokens in the workspace. The workspace also holds
+ * per-slice partial gradients (dk / 32 slices of 32 value columns), which a
+ * second kernel adds in a fixed order, so results are deterministic.
  *   dO              qkv_dtype [B, T, H, dv]
  *   dS_final        fp32 [N, H, dk, dv] or NULL (zero)
  *   grad_q, grad_k  fp32 [B, T, H, dk]       grad_v     fp32 [B, T, H, dv]
