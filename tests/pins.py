@@ -367,6 +367,7 @@ BACKWARD_TOL = {
     "b1_central_differences": 1e-7,
     "b2_varlen_central_differences": 1e-7,
     "b3_pure_decay_closed_form": 1e-12,
+    "b4_chunk_parallel_form": 1e-10,
 }
 
 _GRAD_OF = (("q", "dq"), ("k", "dk"), ("v", "dv"), ("log_alpha", "dlog_alpha"),
@@ -443,10 +444,94 @@ def pin_b3_pure_decay_closed_form(orc):
                     (g["dlog_alpha"][0, :, 0], dla), (g["dk"], 0 * k), (g["dv"], 0 * v))
 
 
+def _chunked_backward(q, k, v, la, beta, S0, dO, dSf, scale, C):
+    """Gradients of one (sequence, head) through the chunk-parallel form of the
+    rule, an independent derivation. In a chunk with entry state S and inclusive
+    cumulative log-decay g (per channel), with E_rs = e^{g_r - g_s} (r >= s):
+        A_rs = beta_r k_r.(E_rs k_s) (s < r),  Pm_rs = q_r.(E_rs k_s) (s <= r),
+        T = (I + A)^{-1},  W = T Diag(beta) (e^g k),  U = T Diag(beta) V - W S,
+        O = scale (e^g q) S + scale Pm U,  S_end = Diag(e^{g_C}) S + (e^{g_C - g} k)^T U.
+    Reverse-mode through these block products, written so that every
+    exponential is an E_rs <= 1. Only e^{g_r - g_s} with r >= s appears, so
+    strong decay cannot overflow."""
+    T_, dk = q.shape
+    n_ch = (T_ + C - 1) // C
+    S = S0.copy()
+    saved = []
+    for c in range(n_ch):
+        a, e = c * C, min(T_, (c + 1) * C)
+        n = e - a
+        g = np.cumsum(la[a:e], axis=0)
+        low = np.tril(np.ones((n, n)))
+        E = np.exp(np.minimum(g[:, None, :] - g[None, :, :], 0.0)) * low[:, :, None]
+        kk = np.einsum("rc,sc,rsc->rs", k[a:e], k[a:e], E) * np.tril(np.ones((n, n)), -1)
+        Pm = np.einsum("rc,sc,rsc->rs", q[a:e], k[a:e], E)
+        Tm = np.linalg.inv(np.eye(n) + beta[a:e, None] * kk)
+        bv = beta[a:e, None] * v[a:e]
+        bk = beta[a:e, None] * k[a:e] * np.exp(g)
+        W = Tm @ bk
+        U = Tm @ bv - W @ S
+        saved.append((a, e, g, E, kk, Pm, Tm, bv, bk, W, U, S.copy()))
+        S = np.exp(g[-1])[:, None] * S + (k[a:e] * np.exp(g[-1] - g)).T @ U
+    G = dSf.copy()
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v),
+               dlog_alpha=np.zeros_like(la), dbeta=np.zeros_like(beta))
+    for a, e, g, E, kk, Pm, Tm, bv, bk, W, U, S in reversed(saved):
+        qc, kc, vc, bc, do = q[a:e], k[a:e], v[a:e], beta[a:e], dO[a:e]
+        eg, egC = np.exp(g), np.exp(g[-1])
+        kh = kc * np.exp(g[-1] - g)
+        dU = scale * Pm.T @ do + kh @ G
+        dPm = np.tril(scale * do @ U.T)
+        dW = -dU @ S.T
+        xv, xk = Tm.T @ dU, Tm.T @ dW
+        dA = np.tril(-Tm.T @ (dU @ bv.T + dW @ bk.T) @ Tm.T, -1)
+        bdA = bc[:, None] * dA
+        X = np.einsum("rs,sc,rsc->rc", dPm, kc, E)
+        Y = np.einsum("rs,rc,rsc->sc", dPm, qc, E)
+        Z = np.einsum("rs,sc,rsc->rc", bdA, kc, E)
+        R = np.einsum("rs,rc,rsc->sc", bdA, kc, E)
+        Kt = np.exp(g[-1] - g) * (U @ G.T)
+        dq = scale * eg * (do @ S.T) + X
+        dk_ = bc[:, None] * eg * xk + Z + Y + R + Kt
+        dg = qc * dq + kc * (dk_ - 2.0 * (Y + R + Kt))
+        dg[-1] += np.sum(kc * Kt, axis=0) + egC * np.sum(G * S, axis=1)
+        out["dq"][a:e], out["dk"][a:e], out["dv"][a:e] = dq, dk_, bc[:, None] * xv
+        out["dbeta"][a:e] = (np.sum(xv * vc, 1) + np.sum(xk * kc * eg, 1) + np.sum(dA * kk, 1))
+        out["dlog_alpha"][a:e] = np.cumsum(dg[::-1], axis=0)[::-1]
+        G = scale * (qc * eg).T @ do + egC[:, None] * G - W.T @ dU
+    out["dS0"] = G
+    return out
+
+
+def pin_b4_chunk_parallel_form(orc):
+    """The backward equals the reverse of the chunk-parallel form (chunks of 16
+    over 150 tokens, so that the oracle's own 64-token replay blocks are crossed
+    too; dk != dv, two heads, with and without strong decay), relative to the
+    largest gradient of each kind."""
+    worst = 0.0
+    for seed, shift in ((107, 0.0), (108, 3.0)):
+        q, k, v, la, b, S0 = _rand(seed, B=1, T=150, H=2, dk=5, dv=4, unit_k=True)
+        la = la * (1.0 + shift)  # at shift 3 the log-decay inside one chunk reaches about -68
+        r = np.random.default_rng(seed + 50)
+        dO, dSf = r.normal(size=v.shape), r.normal(size=S0.shape)
+        scale = 0.45
+        g = orc.backward(q, k, v, la, b, dO, S0, dSf, scale=scale)
+        for h in range(2):
+            ref = _chunked_backward(q[0, :, h], k[0, :, h], v[0, :, h], la[0, :, h], b[0, :, h],
+                                    S0[0, h], dO[0, :, h], dSf[0, h], scale, 16)
+            for key in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+                x, y = g[key][0, :, h], ref[key]
+                worst = max(worst, float(np.abs(x - y).max() / max(1e-30, np.abs(y).max())))
+            x, y = g["dS0"][0, h], ref["dS0"]
+            worst = max(worst, float(np.abs(x - y).max() / max(1e-30, np.abs(y).max())))
+    return worst
+
+
 BACKWARD_ALL = {
     "b1_central_differences": pin_b1_central_differences,
     "b2_varlen_central_differences": pin_b2_varlen_central_differences,
     "b3_pure_decay_closed_form": pin_b3_pure_decay_closed_form,
+    "b4_chunk_parallel_form": pin_b4_chunk_parallel_form,
 }
 
 
