@@ -105,3 +105,24 @@ def test_backward_leaves_tokens_outside_sequences_unwritten():
         assert torch.all(got[:, 70:] == sentinel), key
         assert rel_l2(got[:, :70], ref[key][:, :70]) <= TOL, key
     assert rel_l2(out["dS0"].cpu(), ref["dS0"][:2]) <= TOL
+
+
+@pytest.mark.slow
+def test_backward_bench_shape_sampled_heads():
+    """The benchmark's backward shape and launch configuration (B=1, H=32, T=8192,
+    d=128, bf16 inputs, slow decay; 128 CTAs, 256 replay blocks per CTA). The GPU
+    computes all 32 heads. The oracle checks 8 of them, since heads are independent."""
+    P = I.LONG
+    x = I.make_prefill(1, 8192, P.H, P.d, P.dtype, P.gate_shift, 0.0, P.seed + 1000)
+    g = torch.Generator().manual_seed(P.seed + 7)
+    dO = torch.randn(x["v"].shape, generator=g).to(P.dtype)
+    got = kda.kda_chunk_bwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["log_alpha"].cuda(),
+                            x["beta"].cuda(), dO.cuda(), scale=x["scale"])
+    torch.cuda.synchronize()
+    heads = [0, 4, 9, 13, 18, 22, 27, 31]
+    sel = lambda t: t[:, :, heads].contiguous()
+    ref = oracle.backward(sel(x["q"]), sel(x["k"]), sel(x["v"]), sel(x["log_alpha"]),
+                          sel(x["beta"]), sel(dO), scale=x["scale"])
+    errs = {key: rel_l2(got[key][:, :, heads], ref[key]) for key in KEYS if key != "dS0"}
+    errs["dS0"] = rel_l2(got["dS0"][:, heads], ref["dS0"])
+    assert all(np.isfinite(e) and e <= TOL for e in errs.values()), errs
