@@ -237,7 +237,9 @@ kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v,
  * cores for every supported head size; the states are replayed from
  * checkpoints kept every 32 tokens in the workspace. The workspace also holds
  * per-slice partial gradients (dk / 32 slices of 32 value columns), which a
- * second kernel adds in a fixed order, so results are deterministic.
+ * second kernel adds in a fixed order, so results are deterministic. At
+ * d = 128 it takes about 8.2 KB per token and head plus 2.2 MB per (sequence,
+ * head), e.g. 2.2 GB for B = 1, H = 32, T = 8192.
  *   dO              qkv_dtype [B, T, H, dv]
  *   dS_final        fp32 [N, H, dk, dv] or NULL (zero)
  *   grad_q, grad_k  fp32 [B, T, H, dk]       grad_v     fp32 [B, T, H, dv]
