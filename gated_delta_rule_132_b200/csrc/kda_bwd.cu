@@ -62,12 +62,6 @@ struct BwdParams {
     float4 *blk;                  // [CTAs][kBlk + 1][8 * dk]
 };
 
-template <typename TIn>
-__device__ __forceinline__ float ld(const void *p, size_t i)
-{
-    return to_f32(static_cast<const TIn *>(p)[i]);
-}
-
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
 {
     const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
