@@ -1,18 +1,20 @@
 #!/usr/bin/env python
 """Benchmark of the KDA hot path on B200: long-context prefill tokens/s and
-decode-step state GB/s, each against the HBM roofline.
+decode-step state GB/s, each against its roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One "step" is one chunked prefill of the long-context workload (B=1, H=32,
 T=131072, d=128, bf16 q/k/v, fp32 gates, zero S0): the chunk-parallel kernel
-and the sequential carry kernel. The decode workload (256 sequences x 32 heads,
-128 x 128 fp32 state, bf16 q/k/v) is timed the same way and reported under
-"decode". Inputs are seeded synthetic tensors resident in HBM before the timed
-region; every workload's inputs are larger than the 126 MB L2, so no flush is
-needed between iterations. Under torchrun each rank runs its own independent
-problem (weak scaling, no collective on the data path) and the time is the max
-over ranks.
+and the sequential carry kernel. The other workloads are reported under their
+own keys: the chunked (B=4, H=16, T=4096) and varlen (8 packed sequences) prefills,
+the decode workload (256 sequences x 32 heads, 128 x 128 fp32 state, bf16
+q/k/v) as a chain of 1000 steps with fresh inputs per step, the multi-token
+decode, the one-gate-per-head prefill and the backward. Inputs are seeded
+synthetic tensors resident in HBM before the timed region; every workload's
+inputs are larger than the 126 MB L2, so no flush is needed between
+iterations. Under torchrun each rank runs its own independent problem (weak
+scaling, no collective on the data path) and the time is the max over ranks.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
 bounded sample of the same workload per step (rank 0 only).
@@ -36,16 +38,29 @@ from gated_delta_rule_132_b200 import inputs as I  # noqa: E402
 
 METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM peak, "
           "1×B200")
-# Kernels one tcgen05 prefill call launches: plan, prep, exact fixup (exits at
-# once when no chunk needs it), carry. (The error-word reset is a memset.)
-LAUNCHES_PER_PREFILL = 4
-# DRAM traffic per (chunk, head) record measured by ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum) on the chunked workload, one launch of 4096 records;
-# traffic grows in proportion to the records a launch processes. Sources:
-# profiles/tc_prep2_kernel_chunked_B4_H16_T4096.md,
-# profiles/tc_gdn_prep_kernel_chunked_B4_H16_T4096.md and
-# profiles/tc_carry_kernel_chunked_B4_H16_T4096.md.
+# DRAM traffic per (chunk, head) record (dram__bytes_read.sum +
+# dram__bytes_write.sum of one ncu capture of each kernel on the chunked
+# workload, 4096 records per launch); traffic grows in proportion to the
+# records a launch processes.
 TRAFFIC_PER_RECORD = {"prepare": 162_115, "carry": 105_452, "gdn_prepare": 128_435}
+# Algorithmic work of the prefill per token and head at d = 128, chunk 64: bytes
+# the operation must move (q, k, v bf16 in, log_alpha and beta fp32 in, o bf16
+# out; the states are added per sequence) and tensor-core flops of the chunked
+# form, split into the intra-chunk contractions (A, P and the solve's products:
+# 10 C d) and the inter-chunk state carry (6 d^2).
+PREFILL_IN_BYTES = 3 * 128 * 2 + 128 * 4 + 4
+PREFILL_OUT_BYTES = 128 * 2
+INTRA_FLOP = 10 * 64 * 128
+CARRY_FLOP = 6 * 128 * 128
+# The pages' own claims, quoted as context only: whole-model ratios of Kimi
+# Linear against full attention (no hardware or precision stated).
+PAGE_CLAIMS = {
+    "decode_speed_1M_tokens": "about 6x faster decoding than full attention at 1M tokens",
+    "decode_speedup_128k_1M": "4.8x at 128k and 6.3x at 1M tokens",
+    "kv_cache": "up to 75% less KV cache",
+    "long_context_speed": "2.9x faster on 100k-token long-context work",
+    "note": "whole-model ratios from the pages, not kernel numbers; context only",
+}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -148,18 +163,25 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+LAUNCHES = {"count": 0}  # the library's kernel launches inside every timed region
+
+
 def time_region(fn_step, steps, stream, marks=0):
     """Run ``fn_step(i, events)`` for i < steps between two events on ``stream``.
     ``marks`` extra events per step are handed to fn_step to bracket kernels.
-    Returns (total ms, [[ms between consecutive marks] per step])."""
+    Returns (total ms, [[ms between consecutive marks] per step]); the library's
+    kernel launches inside the region are added to LAUNCHES."""
+    from gated_delta_rule_132_b200 import kda
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(marks)] for _ in range(steps)]
+    n0 = kda.kda_launch_count()
     start.record(stream)
     for i in range(steps):
         fn_step(i, evs[i])
     end.record(stream)
     torch.cuda.synchronize()
+    LAUNCHES["count"] += kda.kda_launch_count() - n0
     per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(marks - 1)]
            for i in range(steps)]
     return start.elapsed_time(end), per
@@ -193,7 +215,9 @@ def bench_prefill(preset, steps, warmup, world, rank, dev, peaks):
         call.carry()
         ev[2].record(stream)
 
+    n0 = LAUNCHES["count"]
     total_ms, per = time_region(step, steps, stream, marks=3)
+    launches = LAUNCHES["count"] - n0
     barrier(world)
     ms = max_over_ranks(total_ms / steps, world)
     prep_ms = statistics.mean(p[0] for p in per)
@@ -201,10 +225,9 @@ def bench_prefill(preset, steps, warmup, world, rank, dev, peaks):
     tokens = x["q"].shape[0] * x["q"].shape[1]
     token_heads = tokens * preset.H
     d = preset.d
-    in_b = 3 * d * x["q"].element_size() + 4 * d + 4     # q,k,v + log_alpha + beta
-    out_b = d * x["q"].element_size()                     # o
-    n_seq = 1 if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
-    n_seq = preset.B if x["cu_seqlens"] is None else n_seq
+    in_b = PREFILL_IN_BYTES                               # q,k,v + log_alpha + beta
+    out_b = PREFILL_OUT_BYTES                             # o
+    n_seq = preset.B if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
     state_b = n_seq * preset.H * d * d * 4 * (2 if x["S0"] is not None else 1)
     op_bytes = token_heads * (in_b + out_b) + state_b
     ws_bytes = call.workspace.numel()
@@ -214,6 +237,7 @@ def bench_prefill(preset, steps, warmup, world, rank, dev, peaks):
         cu = x["cu_seqlens"].cpu().tolist()
         chunks = sum((cu[i + 1] - cu[i] + 63) // 64 for i in range(len(cu) - 1))
     return dict(x=x, call=call, ms=ms, prep_ms=prep_ms, carry_ms=carry_ms, tokens=tokens,
+                launches=launches, n_seq=n_seq,
                 token_heads=token_heads, op_bytes=op_bytes, in_bytes=token_heads * in_b,
                 out_bytes=token_heads * out_b + state_b, ws_bytes=ws_bytes,
                 records=chunks * preset.H)
@@ -293,33 +317,42 @@ def bench_backward(steps, warmup, world, rank, dev, T_b=BWD_T):
                 token_heads=T_b * P.H, workload=f"long_bf16_B1_H{P.H}_T{T_b}_d{P.d}")
 
 
-def bench_decode(P, steps, warmup, world, rank, dev):
+def bench_decode(P, warmup, world, rank, dev):
+    """The decode workload as a chain of P.steps (1000) steps: every step's
+    token inputs (fresh seeded q, k, v and gates per step) are generated on the
+    device before the timed region, the state is carried from step to step,
+    and every step is bracketed by events. GB/s = bytes per step / median step
+    time."""
     from gated_delta_rule_132_b200 import kda
     devs = f"cuda:{dev}"
-    S = I.make_decode_state(P.N, P.H, P.d, P.s_std, P.seed + 1000 * rank, device=devs)
+    S0 = I.make_decode_state(P.N, P.H, P.d, P.s_std, P.seed + 1000 * rank, device=devs)
     toks = [I.make_decode_token(P.N, P.H, P.d, P.dtype, P.gate_shift,
                                 seed=P.step_seed0 + i + 100000 * rank, device=devs)
-            for i in range(warmup + steps)]
+            for i in range(P.steps)]
     o = torch.empty(P.N, P.H, P.d, dtype=P.dtype, device=devs)
+    S = S0.clone()
     stream = torch.cuda.current_stream()
     for i in range(warmup):
         kda.kda_decode_step(**toks[i], S=S, o=o)
+    S.copy_(S0)  # the timed chain starts from the workload's state
     torch.cuda.synchronize()
     barrier(world)
 
     def step(i, ev):
         ev[0].record(stream)
-        kda.kda_decode_step(**toks[warmup + i], S=S, o=o)
+        kda.kda_decode_step(**toks[i], S=S, o=o)
         ev[1].record(stream)
 
-    total_ms, per = time_region(step, steps, stream, marks=2)
+    total_ms, per = time_region(step, P.steps, stream, marks=2)
     barrier(world)
-    ms = max_over_ranks(total_ms / steps, world)
-    kern_ms = statistics.mean(p[0] for p in per)
+    per = [p[0] for p in per]
+    med = max_over_ranks(statistics.median(per), world)
     units = P.N * P.H
     state_b = 2 * units * P.d * P.d * 4
     io_b = units * (3 * P.d * 2 + 4 * P.d + 4 + P.d * 2)
-    return dict(ms=ms, kern_ms=kern_ms, bytes=state_b + io_b, state_bytes=state_b)
+    del toks
+    return dict(ms=max_over_ranks(total_ms / P.steps, world), kern_ms=med, min_ms=min(per),
+                steps=P.steps, bytes=state_b + io_b, state_bytes=state_b)
 
 
 DECODE_TOKENS_T = 8  # tokens per multi-token decode call
@@ -414,43 +447,81 @@ def cpu_baseline(pre_x, preset, budget_s=12.0):
                       f"({dt:.1f} s, fp64 token-by-token, {used} threads)"}
 
 
+def prefill_summary(pre, preset, hbm, tc_peak):
+    """Throughput and roofline figures of one prefill measurement."""
+    kernels = {
+        "prepare": {"ms": pre["prep_ms"], "bytes": pre["in_bytes"],
+                    "flop": pre["token_heads"] * INTRA_FLOP},
+        "carry": {"ms": pre["carry_ms"], "bytes": pre["out_bytes"],
+                  "flop": pre["token_heads"] * CARRY_FLOP},
+    }
+    flop = pre["token_heads"] * (INTRA_FLOP + CARRY_FLOP)
+    op_ach = pre["op_bytes"] / (pre["ms"] / 1e3) / 1e9
+    tc_ach = flop / (pre["ms"] / 1e3) / 1e12
+    return {
+        "workload": preset.name, "tokens": int(pre["tokens"]),
+        "ms_per_step": round(pre["ms"], 4),
+        "kernels_ms": {n: round(v["ms"], 4) for n, v in kernels.items()},
+        "op_roofline": {"bound": "hbm", "achieved": round(op_ach, 1), "peak": hbm,
+                        "unit": "GB/s", "frac": round(op_ach / hbm, 4),
+                        "bytes_per_step": pre["op_bytes"],
+                        "note": "algorithmic bytes of the whole prefill (q,k,v,log_alpha,beta "
+                                "in, o out, states) / step time"},
+        "tc": {"bound": "tensor", "achieved": round(tc_ach, 2), "peak": tc_peak,
+               "unit": "TFLOP/s", "frac": round(tc_ach / tc_peak, 4),
+               "flop_per_token_head": INTRA_FLOP + CARRY_FLOP,
+               "intra_chunk_frac_of_prepare": round(
+                   kernels["prepare"]["flop"] / (kernels["prepare"]["ms"] / 1e3) / 1e12 /
+                   tc_peak, 4),
+               "note": "tensor-core flops of the chunked form / step time, against the "
+                       "sustained bf16 peak"},
+    }, kernels
+
+
 def run_ours(args, world, rank, dev):
     from gated_delta_rule_132_b200 import kda
     kda.lib()
     peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     preset = {"long": I.LONG, "chunked": I.CHUNKED, "varlen": I.VARLEN}[args.workload]
     clocks = ClockSampler(dev)
+    extra = {}
     with clocks:
         pre = bench_prefill(preset, args.steps, args.warmup, world, rank, dev, peaks)
-        dec = None if args.no_decode else bench_decode(I.DECODE, args.steps, args.warmup,
-                                                       world, rank, dev)
+        if not args.no_configs:
+            for other in (I.CHUNKED, I.VARLEN):
+                if other is preset:
+                    continue
+                o = bench_prefill(other, args.config_steps, args.warmup, world, rank, dev, peaks)
+                extra[other.name] = o
+                del o["x"], o["call"]
+                torch.cuda.empty_cache()
+        dec = None if args.no_decode else bench_decode(I.DECODE, args.warmup, world, rank, dev)
         dtok = None if args.no_decode else bench_decode_tokens(
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
         gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
         bwd = None if args.no_backward else bench_backward(
             min(args.steps, 3), args.warmup, world, rank, dev, args.bwd_tokens)
-    hbm = peaks["hbm_gbs"]
     value = job_throughput(pre["tokens"], pre["ms"], world)
+    summ, kernels = prefill_summary(pre, preset, hbm, tc_peak)
 
-    # Dominant prefill kernel and its roofline (HBM: the bytes it must move, i.e.
-    # its inputs plus the per-chunk records it writes (prepare) or reads
-    # (carry) plus its outputs, over its measured time).
-    ws_per_launch = pre["ws_bytes"]
-    prep_bytes = pre["in_bytes"] + ws_per_launch
-    carry_bytes = ws_per_launch + pre["out_bytes"]
-    kernels = {
-        "prepare": {"ms": pre["prep_ms"], "bytes": prep_bytes},
-        "carry": {"ms": pre["carry_ms"], "bytes": carry_bytes},
-    }
+    # Roofline of the dominant prefill kernel: the operation's algorithmic bytes
+    # (1540 B per token and head plus the states) over that kernel's time, and
+    # the DRAM traffic ncu measured for it (per record x records) against its
+    # own algorithmic bytes.
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
-    ach = kernels[dom]["bytes"] / (kernels[dom]["ms"] / 1e3) / 1e9
+    ach = pre["op_bytes"] / (kernels[dom]["ms"] / 1e3) / 1e9
+    traffic = {n: TRAFFIC_PER_RECORD[n] * pre["records"] for n in kernels}
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
-            "unit": "GB/s", "frac": round(ach / hbm, 4),
-            "traffic": TRAFFIC_PER_RECORD[dom] * pre["records"],
-            "traffic_note": "ncu DRAM bytes per record on the chunked workload x records",
+            "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": traffic[dom],
             "peak_source": peak_kind,
-            "bytes_per_launch": kernels[dom]["bytes"], "ms_per_launch": kernels[dom]["ms"]}
-    op_ach = pre["op_bytes"] / (pre["ms"] / 1e3) / 1e9
+            "bytes_per_launch": pre["op_bytes"], "ms_per_launch": round(kernels[dom]["ms"], 4),
+            "note": "algorithmic bytes of the whole prefill / the dominant kernel's time",
+            "traffic_vs_algorithmic": {
+                dom: round(traffic[dom] / kernels[dom]["bytes"], 3),
+                "prefill": round(sum(traffic.values()) / pre["op_bytes"], 3)},
+            "traffic_note": "ncu DRAM bytes per record on the chunked workload x records"}
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["ms"], 4),
@@ -462,24 +533,33 @@ def run_ours(args, world, rank, dev):
                    "l2": "inputs larger than L2 (no flush needed)",
                    "parallelism": f"independent problem per GPU x{world}"},
         "roofline": roof,
-        "op_roofline": {"bound": "hbm", "achieved": round(op_ach, 1), "peak": hbm,
-                        "unit": "GB/s", "frac": round(op_ach / hbm, 4),
-                        "bytes_per_step": pre["op_bytes"],
-                        "note": "algorithmic bytes of the whole prefill (q,k,v,log_alpha,"
-                                "beta in, o out, states) / step time"},
-        "kernels_ms": {n: round(v["ms"], 4) for n, v in kernels.items()},
-        "kernels_roofline_frac": {n: round(v["bytes"] / (v["ms"] / 1e3) / 1e9 / hbm, 4)
-                                  for n, v in kernels.items()},
-        "gpu_launches": LAUNCHES_PER_PREFILL * args.steps,
+        "op_roofline": summ["op_roofline"],
+        "tc": summ["tc"],
+        "kernels_ms": summ["kernels_ms"],
+        "gpu_launches": pre["launches"],
+        "gpu_launches_note": "library kernel launches counted inside the timed prefill "
+                             "region (kda_launch_count)",
     }
+    for name, o in extra.items():
+        sm, _ = prefill_summary(o, I.PRESETS[name], hbm, tc_peak)
+        sm["value"] = round(job_throughput(o["tokens"], o["ms"], world), 1)
+        sm["unit"] = "tokens/s"
+        sm["steps"] = args.config_steps
+        line[name.split("_")[0]] = sm
     if dec is not None:
         dec_ach = dec["bytes"] / (dec["kern_ms"] / 1e3) / 1e9
         line["decode"] = {"workload": I.DECODE.name, "value": round(dec_ach, 1), "unit": "GB/s",
+                          "steps": dec["steps"], "chained": True,
                           "ms_per_step": round(dec["kern_ms"], 4),
+                          "ms_per_step_min": round(dec["min_ms"], 4),
+                          "ms_per_step_mean": round(dec["ms"], 4),
                           "roofline": {"kernel": "decode", "bound": "hbm",
                                        "achieved": round(dec_ach, 1), "peak": hbm,
                                        "unit": "GB/s", "frac": round(dec_ach / hbm, 4),
-                                       "traffic": None, "bytes_per_launch": dec["bytes"]}}
+                                       "frac_of_nominal_8tbs": round(dec_ach / 8000.0, 4),
+                                       "traffic": None, "bytes_per_launch": dec["bytes"]},
+                          "note": "median over the chained steps; inputs of every step "
+                                  "generated on the device before the timed region"}
     if dtok is not None:
         t_ach = dtok["bytes"] / (dtok["kern_ms"] / 1e3) / 1e9
         line["decode_tokens"] = {
@@ -493,18 +573,17 @@ def run_ours(args, world, rank, dev):
                          "frac": round(t_ach / hbm, 4), "traffic": None,
                          "bytes_per_launch": dtok["bytes"]}}
     if gdn is not None:
-        g_ach = (gdn["in_bytes"] + ws_per_launch) / (gdn["prep_ms"] / 1e3) / 1e9
+        g_ach = (gdn["in_bytes"] + pre["out_bytes"]) / (gdn["ms"] / 1e3) / 1e9
         line["gdn"] = {
             "workload": preset.name + "_gate_per_head",
             "value": round(job_throughput(pre["tokens"], gdn["ms"], world), 1),
             "unit": "tokens/s",
             "ms_per_step": round(gdn["ms"], 4),
             "kernels_ms": {"prepare": round(gdn["prep_ms"], 4), "carry": round(gdn["carry_ms"], 4)},
-            "roofline": {"kernel": "prepare (one gate per head)", "bound": "hbm",
-                         "achieved": round(g_ach, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(g_ach / hbm, 4),
-                         "traffic": TRAFFIC_PER_RECORD["gdn_prepare"] * pre["records"],
-                         "bytes_per_launch": gdn["in_bytes"] + ws_per_launch}}
+            "op_roofline": {"bound": "hbm", "achieved": round(g_ach, 1), "peak": hbm,
+                            "unit": "GB/s", "frac": round(g_ach / hbm, 4),
+                            "traffic": TRAFFIC_PER_RECORD["gdn_prepare"] * pre["records"],
+                            "bytes_per_step": gdn["in_bytes"] + pre["out_bytes"]}}
     if bwd is not None:
         tf = bwd["token_heads"] * BWD_FLOP_PER_TOKEN_HEAD / (bwd["kern_ms"] / 1e3) / 1e12
         line["backward"] = {
@@ -518,15 +597,15 @@ def run_ours(args, world, rank, dev):
                          "traffic": BWD_TRAFFIC_PER_TOKEN_HEAD * bwd["token_heads"],
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz",
                          "timed": "whole kda_chunk_bwd call (plan, bwd_kernel, reduction)"}}
-    c = clocks.summary()
-    line["clocks"] = c
+    line["clocks"] = clocks.summary()
     if not args.no_e2e:
-        e = bench_e2e(pre, max(1, min(args.steps, args.e2e_steps)),
-                      torch.cuda.current_stream())
+        e = bench_e2e(pre, max(1, args.e2e_steps), torch.cuda.current_stream())
         e_ms = max_over_ranks(e["ms"], world)
         line["e2e"] = {"value": round(job_throughput(pre["tokens"], e_ms, world), 1),
                        "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
-                       "d2h_bytes_per_step": e["d2h"], "ms_per_step": round(e_ms, 3)}
+                       "d2h_bytes_per_step": e["d2h"], "ms_per_step": round(e_ms, 3),
+                       "steps": max(1, args.e2e_steps)}
+    line["page_claims"] = PAGE_CLAIMS
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(pre["x"], preset)
     if rank == 0:
@@ -589,7 +668,11 @@ def main():
                     help="tokens of the backward measurement (all 32 heads)")
     ap.add_argument("--no-gdn", action="store_true",
                     help="skip the one-gate-per-head (GDN) variant of the prefill")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the chunked and varlen prefill workloads")
+    ap.add_argument("--config-steps", type=int, default=10,
+                    help="timed steps of the chunked and varlen prefill workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=1024,

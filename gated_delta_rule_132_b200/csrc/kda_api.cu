@@ -3,10 +3,28 @@
 // Every check here runs on the host before any launch and touches no device
 // state, so a rejected call has no side effects (and can be made without a GPU).
 #include <math.h>
+#include <stdlib.h>
+
+#include <atomic>
 
 #include "kda_internal.cuh"
 
 namespace {
+
+std::atomic<unsigned long long> g_launches{0};
+std::atomic<uint32_t> g_wait_limit{0};
+std::atomic<int> g_starve_carry{0};
+
+// KDA_DEBUG_SYNC=1 in the environment: every prefill call waits for its work
+// and returns KDA_ERR_DEVICE_STATUS if a bounded wait ran out.
+bool debug_sync()
+{
+    static const bool on = [] {
+        const char *e = getenv("KDA_DEBUG_SYNC");
+        return e != nullptr && e[0] != '\0' && e[0] != '0';
+    }();
+    return on;
+}
 
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool head_ok(int dk, int dv) { return dk == dv && (dk == 32 || dk == 64 || dk == 128); }
@@ -47,7 +65,43 @@ size_t required_bytes(const kda::Problem &p, bool tc) {
 
 }  // namespace
 
+namespace kda {
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+DebugKnobs debug_knobs()
+{
+    return DebugKnobs{g_wait_limit.load(std::memory_order_relaxed),
+                      g_starve_carry.load(std::memory_order_relaxed)};
+}
+
+}  // namespace kda
+
 extern "C" {
+
+unsigned long long kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+kda_status_t kda_debug_set_wait_limit(unsigned int polls, int starve_carry)
+{
+    g_wait_limit.store(polls, std::memory_order_relaxed);
+    g_starve_carry.store(starve_carry ? 1 : 0, std::memory_order_relaxed);
+    return KDA_OK;
+}
+
+kda_status_t kda_chunk_fwd_status(const void *workspace, size_t workspace_bytes,
+                                  int *device_code, void *stream)
+{
+    if (!workspace || !device_code) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGNMENT;
+    if (workspace_bytes < kda::kWsHeader) return KDA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int code = 0;
+    if (cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    *device_code = code;
+    return code != 0 ? KDA_ERR_DEVICE_STATUS : KDA_OK;
+}
 
 const char *kda_status_string(kda_status_t s)
 {
@@ -63,7 +117,7 @@ const char *kda_status_string(kda_status_t s)
     return "unknown status";
 }
 
-int kda_version(void) { return 200; }  // 0.2.0: multi-token decode and the GDN entry points
+int kda_version(void) { return 300; }  // 0.3.0: device status word, launch count
 
 size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
                                        kda_dtype_t dt, int algo)
@@ -116,7 +170,12 @@ static kda_status_t chunk_fwd_phases(const void *q, const void *k, const void *v
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = tc ? kda::launch_tc_prefill(p, workspace, phases, s)
                              : kda::launch_simt_prefill(p, workspace, phases, s);
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    if (debug_sync()) {
+        int code = 0;
+        return kda_chunk_fwd_status(workspace, workspace_bytes, &code, stream);
+    }
+    return KDA_OK;
 }
 
 extern "C" {

@@ -479,10 +479,12 @@ cudaError_t launch_d(const BwdParams &p, float *gq, float *gk, float *gla, float
     if (e != cudaSuccess) return e;
     const unsigned ctas = (unsigned)p.N * p.H * NS;
     kern<<<ctas, Sh::NT, Sh::kBytes, st>>>(p);
+    note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess || p.TH == 0) return e;
     const unsigned grid = (unsigned)std::min<size_t>((p.TH + 7) / 8, (size_t)148 * 32);
     bwd_reduce_kernel<D><<<grid, 256, 0, st>>>(p, NS, gq, gk, gla, gbeta);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -135,6 +135,7 @@ cudaError_t launch_d(const void *q, const void *k, const void *v, const float *l
     decode_kernel<D, D, TIn><<<units, kDecodeThreads, 0, st>>>(
         static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v),
         la, beta, S, T, H, gpc, scale, static_cast<TIn *>(o));
+    note_launch();
     return cudaGetLastError();
 }
 

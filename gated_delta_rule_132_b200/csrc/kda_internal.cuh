@@ -54,6 +54,27 @@ struct Plan {
 // int32 entries of a plan for N sequences.
 inline size_t plan_ints(int N) { return 3 * (size_t)N + 2; }
 
+// Every prefill workspace starts with a header of kWsHeader bytes:
+//   int32 [0]  device status word: 0, or the code of the first bounded wait
+//              that ran out (cleared by the prepare phase; kda_chunk_fwd_status
+//              reads it)
+//   int32 [1]  tensor-core path: number of chunks listed for the exact fixup
+// The plan follows the header.
+constexpr size_t kWsHeader = 256;
+
+// Process-wide debugging settings (kda_debug_set_wait_limit): the poll limit
+// of every bounded wait in the tensor-core kernels (0: the default), and
+// whether the sequential kernel's producer issues no copies, so that its
+// first wait on a record runs out with nothing asynchronous in flight.
+struct DebugKnobs {
+    uint32_t wait_limit;
+    int starve_carry;
+};
+DebugKnobs debug_knobs();
+
+// Counts one kernel launch of this library (kda_launch_count reads the total).
+void note_launch();
+
 // Byte layout of one prefill workspace.
 struct WorkspaceLayout {
     size_t plan_bytes;      // seq_start + chunk_off

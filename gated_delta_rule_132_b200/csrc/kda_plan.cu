@@ -121,6 +121,7 @@ cudaError_t launch_plan(const Problem &p, Plan plan, cudaStream_t stream)
 {
     plan_kernel<<<1, kPlanThreads, 0, stream>>>(p.cu_seqlens, p.N, p.T, (int)p.total_tokens,
                                                 plan.seq_start, plan.chunk_off, plan.order);
+    note_launch();
     return cudaGetLastError();
 }
 

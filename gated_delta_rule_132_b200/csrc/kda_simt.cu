@@ -272,7 +272,7 @@ cudaError_t launch_simt_d(const Problem &pb, void *workspace, int phases, cudaSt
     p.N = pb.N; p.H = pb.H; p.scale = pb.scale; p.o = pb.o; p.S_final = pb.S_final;
     p.gate_per_channel = pb.gate_per_channel;
     Plan plan;
-    plan.seq_start = static_cast<int32_t *>(workspace);
+    plan.seq_start = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
     plan.chunk_off = plan.seq_start + (pb.N + 1);
     plan.order = plan.chunk_off + (pb.N + 1);
     p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off; p.order = plan.order;
@@ -286,16 +286,21 @@ cudaError_t launch_simt_d(const Problem &pb, void *workspace, int phases, cudaSt
     e = cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)carry_smem<D>());
     if (e != cudaSuccess) return e;
     if (phases & kPhasePrepare) {
+        // the status word: this path has no bounded waits, so it stays 0
+        e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+        if (e != cudaSuccess) return e;
         e = launch_plan(pb, plan, st);
         if (e != cudaSuccess) return e;
         if (pb.max_chunks > 0) {
             prep<<<dim3(pb.max_chunks, pb.H), kSimtThreads, prep_smem<D>(), st>>>(p);
+            note_launch();
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
     }
     if (phases & kPhaseCarry) {
         carry<<<(unsigned)(pb.N * pb.H * (D / kSimtSlice)), kSimtThreads, carry_smem<D>(), st>>>(p);
+        note_launch();
         e = cudaGetLastError();
     }
     return e;
@@ -317,7 +322,7 @@ cudaError_t launch_simt_t(const Problem &p, void *ws, int ph, cudaStream_t st)
 WorkspaceLayout simt_workspace_layout(const Problem &p)
 {
     WorkspaceLayout l;
-    l.plan_bytes = align_up(sizeof(int32_t) * plan_ints(p.N), 256);
+    l.plan_bytes = kWsHeader + align_up(sizeof(int32_t) * plan_ints(p.N), 256);
     const size_t D = (size_t)p.dk;
     l.chunk_bytes = sizeof(float) * (4 * C * D + C * C + D) * (size_t)p.H * (size_t)p.max_chunks;
     l.total = l.plan_bytes + l.chunk_bytes;

@@ -86,8 +86,10 @@ struct TcParams {
     float *S_final;
     const int32_t *seq_start, *chunk_off, *order;
     uint8_t *rec;      // records
-    int *err;          // device error word (pipeline timeouts)
+    int *err;          // device status word (the code of the first wait that ran out)
     int *fix_count;    // number of chunks listed for the exact fixup
+    uint32_t spin;     // poll limit of every bounded wait
+    int starve;        // debugging: the carry's producer issues no copies
     int *fix_list;     // chunk * H + head, one per listed chunk
     // q, k, v and log_alpha as 3-D tensors {channel, head, token} for TMA tile
     // loads of 128 bytes of channels x 1 head x 64 tokens in the 128-byte
@@ -502,6 +504,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         tc::mbar_init(bar_ap, 1);
         tc::mbar_init(bar_wu, 1);
         tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(bar_ld + 1, 1);  // bar_fin
         *abort = 0;
         tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_ld, 10 * 8192);
@@ -522,7 +525,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     uint4 qv[4], kv[4], vv[4];
     float g[4][8];
     __syncthreads();  // the barriers are initialised
-    tc::mbar_wait(bar_ld, 0, abort, p.err, 10);
+    tc::mbar_wait(bar_ld, 0, abort, p.err, 10, p.spin);
     {
         float run[8];
 #pragma unroll
@@ -711,7 +714,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     {
         // every warp reads its 32 TMEM lanes; warps 0-3 take the first 32 of the
         // row's 64 relevant columns, warps 4-7 the other 32
-        tc::mbar_wait(bar_ap, 0, abort, p.err, 11);
+        tc::mbar_wait(bar_ap, 0, abort, p.err, 11, p.spin);
         tc::tc_fence_after_sync();
         const int t = (warp & 3) * 32 + (tid & 31);  // accumulator row
         const int sh = (warp >> 2) * 32;             // first s of this thread
@@ -811,7 +814,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
         // Both as record images in the A / T scratch, dead by now: W rows of
         // K-block kb at 8K kb, U~^T at 16K.
-        tc::mbar_wait(bar_wu, 0, abort, p.err, 12);
+        tc::mbar_wait(bar_wu, 0, abort, p.err, 12, p.spin);
         tc::tc_fence_after_sync();
         const int lg = warp & 3, wh = warp >> 2;
         const int row = lg * 32 + (tid & 31);
@@ -848,8 +851,14 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         tc::bulk_s2g(rec + Record::kU, sm + 16384, 32768);
         tc::bulk_commit();
         tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
+        // drain (matters only after a wait gave up): the input tiles have
+        // landed and every MMA has finished before the memory is released
+        tc::mbar_drain(bar_ld, 0, p.err, 13, p.spin);
+        tc::mma_commit(bar_ld + 1);
+        tc::mbar_drain(bar_ld + 1, 0, p.err, 13, p.spin);
     }
     if (warp == 0) {
+        __syncwarp();
         tc::tc_fence_after_sync();
         tc::tmem_dealloc(tmem, 256);
     }
@@ -921,6 +930,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         tc::mbar_init(bar_ap, 1);
         tc::mbar_init(bar_wu, 1);
         tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(bar_ld + 1, 1);  // bar_fin
         *abort = 0;
         tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_ld, 6 * 8192);
@@ -950,7 +960,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
     }
     // rows past the chunk's end (the next sequence, or past the tensor) read zero
     __syncthreads();  // the barriers are initialised
-    tc::mbar_wait(bar_ld, 0, abort, p.err, 20);
+    tc::mbar_wait(bar_ld, 0, abort, p.err, 20, p.spin);
     for (int i = tid; i < 6 * (C - L) * 8; i += kGdnThreads) {
         const int tile = i / ((C - L) * 8), rem = i % ((C - L) * 8);
         const int r = L + (rem >> 3);
@@ -1007,7 +1017,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
     float *Ts = reinterpret_cast<float *>(sm + GdnSmem::kT);
     float *Ys = reinterpret_cast<float *>(sm + GdnSmem::kY);
     {
-        tc::mbar_wait(bar_ap, 0, abort, p.err, 21);
+        tc::mbar_wait(bar_ap, 0, abort, p.err, 21, p.spin);
         tc::tc_fence_after_sync();
         const int t = (warp & 3) * 32 + lane;  // accumulator row
         const int sh = (warp >> 2) * 32;       // first column s of this thread
@@ -1111,7 +1121,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
         // Both as record images in the [K; Q] and V buffers, dead once the MMAs
         // are done: W rows of K-block kb at 8K kb, U~^T at 16K.
-        tc::mbar_wait(bar_wu, 0, abort, p.err, 22);
+        tc::mbar_wait(bar_wu, 0, abort, p.err, 22, p.spin);
         tc::tc_fence_after_sync();
         const int lg = warp & 3, wh = warp >> 2;
         const int row = lg * 32 + lane;
@@ -1148,8 +1158,14 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         tc::bulk_s2g(rec + Record::kU, sm + 16384, 32768);
         tc::bulk_commit();
         tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
+        // drain (matters only after a wait gave up): the input tiles have
+        // landed and every MMA has finished before the memory is released
+        tc::mbar_drain(bar_ld, 0, p.err, 23, p.spin);
+        tc::mma_commit(bar_ld + 1);
+        tc::mbar_drain(bar_ld + 1, 0, p.err, 23, p.spin);
     }
     if (warp == 0) {
+        __syncwarp();
         tc::tc_fence_after_sync();
         tc::tmem_dealloc(tmem, 256);
     }
@@ -1182,7 +1198,7 @@ constexpr int kCarryThreads = 320;
 constexpr int kCarrySync = 288;      // state warps + the MMA warp
 constexpr uint32_t kTmemCols = 512;  // D1[0]: [0,128), D1[1]: [128,256), D2: [256,384)
 
-enum { kErrFull = 1, kErrEmpty, kErrD1, kErrD2, kErrO };
+enum { kErrFull = 1, kErrEmpty, kErrD1, kErrD2, kErrO, kErrDrain };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads)
 {
@@ -1202,6 +1218,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     uint64_t *o_ready = bars + 6;  // MMA3 completed: D1[c & 1] holds O^T of chunk c
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
     volatile int *abort = reinterpret_cast<volatile int *>(bars + 8);
+    uint64_t *drain = bars + 9;    // all MMAs of the CTA completed
 
     // one CTA per (sequence, head, half), sequences longest first
     const int H = p.H;
@@ -1214,6 +1231,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         tc::mbar_init(&full[0], 1); tc::mbar_init(&full[1], 1);
         tc::mbar_init(&empty[0], 9); tc::mbar_init(&empty[1], 9);
         tc::mbar_init(d1_done, 1); tc::mbar_init(d2_done, 1); tc::mbar_init(o_ready, 1);
+        tc::mbar_init(drain, 1);
         *abort = 0;
         tc::fence_mbar_init();
     }
@@ -1229,9 +1247,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     if (warp == 8) {
         // ---------------- producer: one record per chunk into the two-stage ring
         if (lane == 0) {
-            for (int lc = 0; lc < nc; ++lc) {
+            int issued = 0;
+            for (int lc = 0; lc < nc && !p.starve; ++lc) {
                 const int st = lc & 1;
-                if (lc >= 2) tc::mbar_wait(&empty[st], ((lc >> 1) - 1) & 1, abort, p.err, kErrEmpty);
+                if (lc >= 2 && !tc::mbar_wait(&empty[st], ((lc >> 1) - 1) & 1, abort, p.err,
+                                              kErrEmpty, p.spin))
+                    break;
+                if (*abort) break;
                 const uint8_t *rec = p.rec + ((size_t)(c0 + lc) * H + h) * Record::kBytes;
                 uint8_t *sb = sm + st * CarrySmem::kStage;
                 tc::mbar_arrive_expect_tx(&full[st], 32768 + 16384 + 8192 + 16384 + 512);
@@ -1240,10 +1262,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
                 tc::bulk_g2s(sb + CarrySmem::kP, rec + Record::kP, 8192, &full[st]);
                 tc::bulk_g2s(sb + CarrySmem::kU, rec + Record::kU + half * 16384, 16384, &full[st]);
                 tc::bulk_g2s(sb + CarrySmem::kG, rec + Record::kG, 512, &full[st]);
+                issued = lc + 1;
             }
-            // every issued copy has landed before the CTA may exit
-            for (int lc = (nc > 2 ? nc - 2 : 0); lc < nc; ++lc)
-                tc::mbar_wait(&full[lc & 1], (lc >> 1) & 1, abort, p.err, kErrFull);
+            // every issued copy has landed before the CTA may exit (also after
+            // an abort: the copies write this CTA's shared memory)
+            for (int lc = (issued > 2 ? issued - 2 : 0); lc < issued; ++lc)
+                tc::mbar_drain(&full[lc & 1], (lc >> 1) & 1, p.err, kErrFull, p.spin);
         }
     } else if (warp == 9) {
         // ---------------- MMA issue
@@ -1252,14 +1276,20 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         const uint32_t id3 = tc::idesc_bf16(64, 64, 0, 0);   // U^T . P^T
         const uint32_t a_s = tc::smem_u32(sm + CarrySmem::kSt);
         const uint32_t a_u = tc::smem_u32(sm + CarrySmem::kUt);
+        bool issued = false;
         for (int lc = 0; lc < nc; ++lc) {
             const int st = lc & 1;
             const uint32_t sb = tc::smem_u32(sm + st * CarrySmem::kStage);
             const uint32_t d1 = tmem + (uint32_t)st * 128;
-            if (lane == 0) tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
+            // after an abort no MMA is issued; the barriers are still met
+            bool go = false;
+            if (lane == 0)
+                go = tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull, p.spin) &&
+                     !*abort;
             __syncwarp();
             named_bar(1, kCarrySync);  // S^T complete
-            if (lane == 0) {
+            if (go) {
+                issued = true;
                 tc::tc_fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -1270,7 +1300,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             }
             __syncwarp();
             named_bar(2, kCarrySync);  // U^T complete
-            if (lane == 0) {
+            if (go && !*abort) {
                 tc::tc_fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
@@ -1286,6 +1316,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             }
             __syncwarp();
         }
+        // every MMA this thread issued has finished before TMEM is released
+        if (lane == 0 && issued) {
+            tc::mma_commit(drain);
+            tc::mbar_drain(drain, 0, p.err, kErrDrain, p.spin);
+        }
+        __syncwarp();
     } else {
         // ---------------- state owners
         const int lg = warp & 3, wh = warp >> 2, hl = lane >> 4;
@@ -1319,7 +1355,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         uint8_t *os = sm + CarrySmem::kOs + warp * 1024;
         float ov[16];
         auto read_o = [&](int lc) {
-            tc::mbar_wait(o_ready, lc & 1, abort, p.err, kErrO);
+            tc::mbar_wait(o_ready, lc & 1, abort, p.err, kErrO, p.spin);
             tc::tc_fence_after_sync();
             tc::tmem_ld16x2_x16_sync(lane_base + (uint32_t)(lc & 1) * 128 + 64 + 32 * wh, ov);
         };
@@ -1361,8 +1397,8 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             // B. previous chunk's output, while MMA1 runs
             if (lc > 0) store_o(lc - 1);
             // C. U^T = U~^T - (W S)^T for tokens tk0..tk0+15
-            tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull);
-            tc::mbar_wait(d1_done, lc & 1, abort, p.err, kErrD1);
+            tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull, p.spin);
+            tc::mbar_wait(d1_done, lc & 1, abort, p.err, kErrD1, p.spin);
             tc::tc_fence_after_sync();
             {
                 float U[16];
@@ -1394,7 +1430,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
                     const float4 x = *reinterpret_cast<const float4 *>(sb + CarrySmem::kG + (kc0 + j) * 4);
                     g[j] = x.x; g[j + 1] = x.y; g[j + 2] = x.z; g[j + 3] = x.w;
                 }
-                tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2);
+                tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2, p.spin);
                 tc::tc_fence_after_sync();
                 float ku[32];
                 tc::tmem_ld16x2_x32_sync(lane_base + 256 + 64 * wh, ku);
@@ -1471,9 +1507,9 @@ bool tc_supported(const Problem &p)
 WorkspaceLayout tc_workspace_layout(const Problem &p)
 {
     WorkspaceLayout l;
-    // plan arrays, the error word, the fixup count and the fixup list
-    l.plan_bytes = align_up(sizeof(int32_t) * (plan_ints(p.N) + 2 +
-                                               (size_t)p.max_chunks * p.H), 1024);
+    // header (status word, fixup count), plan arrays and the fixup list
+    l.plan_bytes = align_up(kWsHeader + sizeof(int32_t) * (plan_ints(p.N) +
+                                                           (size_t)p.max_chunks * p.H), 1024);
     l.chunk_bytes = (size_t)Record::kBytes * (size_t)p.H * (size_t)p.max_chunks;
     l.total = l.plan_bytes + l.chunk_bytes;
     return l;
@@ -1490,14 +1526,17 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
     p.N = pb.N; p.H = pb.H; p.scale = pb.scale;
     p.o = static_cast<__nv_bfloat16 *>(pb.o); p.S_final = pb.S_final;
     Plan plan;
-    plan.seq_start = static_cast<int32_t *>(workspace);
+    p.err = static_cast<int32_t *>(workspace);
+    p.fix_count = p.err + 1;
+    plan.seq_start = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
     plan.chunk_off = plan.seq_start + (pb.N + 1);
     plan.order = plan.chunk_off + (pb.N + 1);
     p.seq_start = plan.seq_start; p.chunk_off = plan.chunk_off; p.order = plan.order;
-    p.err = plan.order + pb.N;
-    p.fix_count = p.err + 1;
-    p.fix_list = p.err + 2;
+    p.fix_list = plan.order + pb.N;
     p.rec = static_cast<uint8_t *>(workspace) + lay.plan_bytes;
+    const DebugKnobs dbg = debug_knobs();
+    p.spin = dbg.wait_limit ? dbg.wait_limit : tc::kSpinLimit;
+    p.starve = dbg.starve_carry;
 
     cudaError_t e = cudaSuccess;
     if (phases & kPhasePrepare) {
@@ -1517,6 +1556,7 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
                                      (int)GdnSmem::kBytes);
             if (e != cudaSuccess) return e;
             tc_gdn_prep_kernel<<<dim3(pb.max_chunks, pb.H), kGdnThreads, GdnSmem::kBytes, st>>>(p);
+            note_launch();
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         } else if (pb.max_chunks > 0) {
@@ -1524,12 +1564,14 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
                                      (int)Prep2Smem::kBytes);
             if (e != cudaSuccess) return e;
             tc_prep2_kernel<<<dim3(pb.max_chunks, pb.H), kPrep2Threads, Prep2Smem::kBytes, st>>>(p);
+            note_launch();
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
             e = cudaFuncSetAttribute(tc_prep_fixup_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
             if (e != cudaSuccess) return e;
             tc_prep_fixup_kernel<<<kFixupBlocks, kPrepThreads, kPrepSmem, st>>>(p);
+            note_launch();
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
@@ -1539,6 +1581,7 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
                                  (int)CarrySmem::kBytes);
         if (e != cudaSuccess) return e;
         tc_carry_kernel<<<(unsigned)(pb.N * pb.H * kSlices), kCarryThreads, CarrySmem::kBytes, st>>>(p);
+        note_launch();
         e = cudaGetLastError();
     }
     return e;

@@ -55,21 +55,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Spin limit for every wait: far beyond any legitimate wait (each try_wait
-// itself blocks for a while), so only a broken pipeline ever reaches it.
+// Default spin limit for every wait: far beyond any legitimate wait (each
+// try_wait itself blocks for a while), so only a broken pipeline ever reaches
+// it. Kernels take the limit as a parameter so a test can shorten it.
 constexpr uint32_t kSpinLimit = 1u << 20;
 
-// Wait for the phase with the given parity to complete. Gives up after
-// kSpinLimit polls or as soon as *abort is set; on giving up it raises *abort
-// and records `code` in *err (first writer wins) and returns false.
+// Wait for the phase with the given parity to complete. Gives up after `limit`
+// polls or as soon as *abort is set; on giving up it raises *abort, records
+// `code` in *err (first writer wins) and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *err, int code)
+                                          int *err, int code, uint32_t limit = kSpinLimit)
 {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
     }
     *abort = 1;
+    if (err) atomicCAS(err, 0, code);
+    return false;
+}
+
+// Wait for the phase with the given parity to complete, ignoring the abort
+// flag: used to drain asynchronous work this thread issued (copies into shared
+// memory, MMAs) before the CTA releases the memory they use. Gives up after
+// `limit` polls, recording `code`.
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, int *err, int code,
+                                           uint32_t limit = kSpinLimit)
+{
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
     if (err) atomicCAS(err, 0, code);
     return false;
 }

@@ -51,6 +51,12 @@ def lib() -> ctypes.CDLL:
         L.kda_status_string.argtypes = [_i]
         L.kda_version.restype = _i
         L.kda_version.argtypes = []
+        L.kda_launch_count.restype = ctypes.c_ulonglong
+        L.kda_launch_count.argtypes = []
+        L.kda_chunk_fwd_status.restype = _i
+        L.kda_chunk_fwd_status.argtypes = [_vp, _sz, ctypes.POINTER(_i), _vp]
+        L.kda_debug_set_wait_limit.restype = _i
+        L.kda_debug_set_wait_limit.argtypes = [ctypes.c_uint, _i]
         L.kda_chunk_fwd_workspace_size.restype = _sz
         L.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
         L.kda_chunk_fwd_workspace_size_ex.restype = _sz
@@ -184,6 +190,31 @@ class ChunkFwdCall:
 
     def carry(self, stream=None):
         return self._call("kda_chunk_fwd_carry", stream)
+
+
+def kda_launch_count() -> int:
+    """Kernels the library has launched in this process (C: ``kda_launch_count``)."""
+    return int(lib().kda_launch_count())
+
+
+def kda_chunk_fwd_status(workspace: torch.Tensor, stream=None):
+    """Device status word of the last prefill that used ``workspace`` (C:
+    ``kda_chunk_fwd_status``; waits for the stream). Returns ``(status, code)``:
+    status 0 (KDA_OK) with code 0, or 6 (KDA_ERR_DEVICE_STATUS) with the code of
+    the first bounded wait that ran out."""
+    code = _i(0)
+    st = lib().kda_chunk_fwd_status(_p(workspace), workspace.numel() * workspace.element_size(),
+                                    ctypes.byref(code), _stream(stream))
+    if st not in (0, 6):
+        raise KdaError("kda_chunk_fwd_status", st)
+    return st, code.value
+
+
+def kda_debug_set_wait_limit(polls: int = 0, starve_carry: bool = False) -> None:
+    """Debugging aid (C: ``kda_debug_set_wait_limit``): poll limit of the
+    tensor-core kernels' bounded waits (0: default) and whether the sequential
+    kernel's copy producer issues nothing."""
+    lib().kda_debug_set_wait_limit(int(polls), 1 if starve_carry else 0)
 
 
 def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None,

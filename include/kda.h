@@ -37,7 +37,13 @@
  *
  * Errors. Arguments are checked on the host before anything is launched; a bad
  * argument returns an error status and launches nothing. A failed launch returns
- * KDA_ERR_CUDA. The library never aborts, exits or traps.
+ * KDA_ERR_CUDA. The library never aborts, exits or traps. Every wait inside the
+ * tensor-core kernels is bounded; a wait that runs out makes the kernel return
+ * early and records a nonzero code in the prefill workspace's status word, so
+ * the results of that call are not valid. The word is read by
+ * kda_chunk_fwd_status (after the call) or, with KDA_DEBUG_SYNC=1 in the
+ * environment, by every prefill call itself, which then waits for its work and
+ * returns KDA_ERR_DEVICE_STATUS.
  */
 #ifndef KDA_B200_H
 #define KDA_B200_H
@@ -56,7 +62,7 @@ typedef enum {
     KDA_ERR_ALIGNMENT = 3,     /* a buffer is not 16-byte aligned */
     KDA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
     KDA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
-    KDA_ERR_DEVICE_STATUS = 6  /* the device reported an out-of-domain input */
+    KDA_ERR_DEVICE_STATUS = 6  /* a kernel gave up a bounded wait: results invalid */
 } kda_status_t;
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype_t;
@@ -73,6 +79,37 @@ const char *kda_status_string(kda_status_t status);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int kda_version(void);
+
+/* Number of kernels this library has launched in this process so far (all
+ * entry points, all devices). Differences of two readings count the launches
+ * of the calls made in between. */
+unsigned long long kda_launch_count(void);
+
+/*
+ * Device status of the last prefill that used `workspace` (any kda_*chunk_fwd*
+ * entry point, either phase). The library defines no counterpart on the pages;
+ * it reports whether the kernels' own failure detection fired. Reads the
+ * workspace's status word on `stream` and waits for the stream. The prepare
+ * phase clears the word; a later failure in either phase sets it to a nonzero
+ * code (the first failing wait's), which stays until the next prepare.
+ *   workspace, workspace_bytes  the prefill's workspace (>= 256 bytes)
+ *   device_code                 receives the word (0: no wait ran out)
+ * Returns KDA_OK, KDA_ERR_DEVICE_STATUS when the word is nonzero, or an
+ * argument / CUDA error.
+ */
+kda_status_t kda_chunk_fwd_status(const void *workspace, size_t workspace_bytes,
+                                  int *device_code, void *stream);
+
+/*
+ * Debugging aid for the failure path (process-wide; not needed in normal use):
+ * `polls` replaces the poll limit of every bounded wait in the tensor-core
+ * kernels launched afterwards (0 restores the default of 2^20 polls), and a
+ * nonzero `starve_carry` makes the sequential kernel's copy producer issue no
+ * copies, so that its first wait on a chunk record runs out while nothing
+ * asynchronous is in flight. The kernels then return early and the status word
+ * reports the failure. Always returns KDA_OK.
+ */
+kda_status_t kda_debug_set_wait_limit(unsigned int polls, int starve_carry);
 
 /*
  * Workspace bytes that kda_chunk_fwd needs for this problem, i.e. for the path
@@ -279,12 +316,18 @@ kda_status_t kda_gdn_chunk_bwd(const void *q, const void *k, const void *v,
  * device memory, held by every GPU that loads the library until the process
  * exits. The caller still provides every input and output buffer. The call
  * allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
- *   - Problems whose workspace (kda_chunk_fwd_workspace_size) exceeds
+ *   - Problems whose workspace for the same algo
+ *     (kda_chunk_fwd_workspace_size_ex with this call's algo) exceeds
  *     KDA_NOALLOC_SCRATCH_BYTES are rejected on the host with
- *     KDA_ERR_WORKSPACE before anything is launched.
- *   - The first call on each device looks up the scratch array's device
- *     address (cudaGetSymbolAddress, with that device current); make that
- *     first call before any stream capture on the device.
+ *     KDA_ERR_WORKSPACE before anything is launched; invalid arguments are
+ *     rejected on the host as kda_chunk_fwd_ex rejects them.
+ *   - The first call on each device (and the first after the device's
+ *     context was reset) looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture on the device.
+ *   - With KDA_DEBUG_SYNC=1 in the environment the call waits for its work
+ *     and reports a bounded wait that ran out as KDA_ERR_DEVICE_STATUS, as
+ *     kda_chunk_fwd_ex does.
  *   - Every call shares the one array and leaves its contents behind. The
  *     kernels initialise every part of it they read, so nothing carries over
  *     from one call to the next; but calls whose execution overlaps on the GPU

@@ -13,9 +13,50 @@ def rel_l2(x, ref) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
+def _np(x):
+    return np.asarray(x.detach().double().cpu().numpy() if hasattr(x, "detach") else x,
+                      dtype=np.float64)
+
+
+def _ratio(num, den):
+    return np.where(den > 0, num / np.where(den > 0, den, 1.0), num)
+
+
+def unit_errors_o(x, ref, cu_seqlens=None):
+    """Relative L2 error of an output o [B, T, H, d] per (sequence, head), so
+    that a fault confined to one unit is not diluted by the others. Without
+    ``cu_seqlens`` the units are the batch rows; with it (B = 1) sequence n owns
+    the packed tokens cu[n]..cu[n+1]. Returns [sequences, H] (a unit with a
+    zero reference reports its absolute error)."""
+    x, ref = _np(x), _np(ref)
+    if cu_seqlens is None:
+        num = np.sqrt(((x - ref) ** 2).sum(axis=(1, 3)))
+        return _ratio(num, np.sqrt((ref ** 2).sum(axis=(1, 3))))
+    cu = [int(c) for c in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    rows = []
+    for n in range(len(cu) - 1):
+        a, b = x[0, cu[n]:cu[n + 1]], ref[0, cu[n]:cu[n + 1]]
+        rows.append(_ratio(np.sqrt(((a - b) ** 2).sum(axis=(0, 2))),
+                           np.sqrt((b ** 2).sum(axis=(0, 2)))))
+    return np.array(rows)
+
+
+def unit_errors_S(x, ref):
+    """Relative L2 error of a state [N, H, dk, dv] per (sequence, head)."""
+    x, ref = _np(x), _np(ref)
+    num = np.sqrt(((x - ref) ** 2).sum(axis=(2, 3)))
+    return _ratio(num, np.sqrt((ref ** 2).sum(axis=(2, 3))))
+
+
 # Tolerances on relative L2 error against the fp64 oracle: fp32 inputs and
 # bf16 q/k/v (with fp32 gates and state).
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+# Regression guard for the tensor-core prefill on the full-size bf16 workloads:
+# about twice the global relative error measured for o and S_final. It is not
+# a tolerance (that is TOL); it flags a precision regression that would still
+# pass TOL.
+REGRESSION_GUARD = {"o": 8e-3, "S": 6e-3}
 
 
 def to_cuda(d):

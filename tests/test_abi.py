@@ -189,3 +189,23 @@ def test_workspace_size_per_algorithm(L):
     assert L.kda_chunk_fwd_workspace_size(1, 4096, 8, 128, 128, 0, 1) == tc
     assert L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 64, 64, 0, 1, 2) == 0
     assert L.kda_chunk_fwd_workspace_size_ex(1, 4096, 8, 128, 128, 0, 1, 7) == 0
+
+
+def test_status_query_rejects_bad_arguments(L):
+    """kda_chunk_fwd_status checks its arguments on the host (no CUDA call)."""
+    code = ctypes.c_int(0)
+    assert L.kda_chunk_fwd_status(None, 1024, ctypes.byref(code), None) == 1
+    assert L.kda_chunk_fwd_status(_fake(), 1024, None, None) == 1
+    assert L.kda_chunk_fwd_status(_fake(0x10004), 1024, ctypes.byref(code), None) == 3
+    assert L.kda_chunk_fwd_status(_fake(), 255, ctypes.byref(code), None) == 4
+
+
+def test_launch_count_and_debug_knobs(L):
+    """The launch counter starts at a number and rejected calls launch nothing;
+    the debug knobs accept any value and are reset."""
+    L.kda_launch_count.restype = ctypes.c_ulonglong
+    before = L.kda_launch_count()
+    assert _chunk(L, q=None) == 1
+    assert L.kda_launch_count() == before
+    assert L.kda_debug_set_wait_limit(1000, 1) == 0
+    assert L.kda_debug_set_wait_limit(0, 0) == 0

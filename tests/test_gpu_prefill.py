@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import oracle
-from common import TOL, rel_l2, to_cuda
+from common import REGRESSION_GUARD, TOL, rel_l2, to_cuda, unit_errors_o, unit_errors_S
 from gated_delta_rule_132_b200 import inputs as I
 from gated_delta_rule_132_b200 import kda
 
@@ -134,34 +134,49 @@ def test_deterministic_and_in_place_state(algo):
     assert torch.equal(o3, o1) and torch.equal(S, S1)
 
 
+def check_full_size(o, Sf, o_ref, S_ref, cu_seqlens=None):
+    """Every (sequence, head) unit within the bf16 tolerance on its own (a fault
+    in one unit is not diluted by the others), the whole tensors within it too,
+    and the global errors within the regression guard (about twice the errors
+    measured for the tensor-core path; not a tolerance)."""
+    eo = unit_errors_o(o, o_ref, cu_seqlens)
+    eS = unit_errors_S(Sf, S_ref)
+    assert eo.max() <= TOL[torch.bfloat16], f"worst (sequence, head) of o: {eo.max():.3e}"
+    assert eS.max() <= TOL[torch.bfloat16], f"worst (sequence, head) of S: {eS.max():.3e}"
+    go, gS = rel_l2(o, o_ref), rel_l2(Sf, S_ref)
+    assert go <= TOL[torch.bfloat16] and gS <= TOL[torch.bfloat16]
+    assert go <= REGRESSION_GUARD["o"], f"o error {go:.3e} regressed"
+    assert gS <= REGRESSION_GUARD["S"], f"S_final error {gS:.3e} regressed"
+
+
 def test_chunked_config_full_size():
-    """B=4, H=16, T=4096, d=128, bf16, S0 ~ N(0, 0.01): every output checked."""
+    """B=4, H=16, T=4096, d=128, bf16, S0 ~ N(0, 0.01): every output checked,
+    each of the 64 (sequence, head) units on its own."""
     x = I.make_preset(I.CHUNKED)
     o, Sf, o_ref, S_ref = run_both(x)
-    assert rel_l2(o, o_ref) <= 2e-2
-    assert rel_l2(Sf, S_ref) <= 2e-2
+    check_full_size(o, Sf, o_ref, S_ref)
 
 
 @pytest.mark.slow
 def test_long_context_config_sampled_heads():
     """B=1, H=32, T=131072, d=128, bf16, slow decay: the GPU runs all 32 heads;
-    the oracle checks 4 of them end to end (heads are independent)."""
+    the oracle checks 8 of them end to end (heads are independent), each on its
+    own."""
     x = I.make_preset(I.LONG)
-    heads = [0, 9, 21, 31]
+    heads = [0, 4, 9, 13, 18, 21, 26, 31]
     o, Sf, o_ref, S_ref = run_both(x, heads=heads)
-    assert rel_l2(o, o_ref) <= 2e-2
-    assert rel_l2(Sf, S_ref) <= 2e-2
+    check_full_size(o, Sf, o_ref, S_ref)
 
 
 @pytest.mark.slow
 def test_varlen_config_sampled_heads():
     """8 packed sequences of seeded lengths in [1024, 65536], H=32, d=128, bf16,
-    per-sequence S0: the oracle checks every sequence on 3 heads."""
+    per-sequence S0: the oracle checks every sequence on 3 heads, each
+    (sequence, head) on its own."""
     x = I.make_preset(I.VARLEN)
     heads = [2, 17, 30]
     o, Sf, o_ref, S_ref = run_both(x, heads=heads)
-    assert rel_l2(o, o_ref) <= 2e-2
-    assert rel_l2(Sf, S_ref) <= 2e-2
+    check_full_size(o, Sf, o_ref, S_ref, cu_seqlens=x["cu_seqlens"])
 
 
 @pytest.mark.parametrize("algo", ["simt", "tcgen05"])
