@@ -41,8 +41,8 @@ METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM pea
 # DRAM traffic per (chunk, head) record (dram__bytes_read.sum +
 # dram__bytes_write.sum of one ncu capture of each kernel on the chunked
 # workload, 4096 records per launch); traffic grows in proportion to the
-# records a launch processes.
-TRAFFIC_PER_RECORD = {"prepare": 162_115, "carry": 105_452, "gdn_prepare": 128_435}
+# records a launch processes. None: no capture of the current kernel yet.
+TRAFFIC_PER_RECORD = {"prepare": None, "carry": None, "gdn_prepare": None}
 # Algorithmic work of the prefill per token and head at d = 128, chunk 64: bytes
 # the operation must move (q, k, v bf16 in, log_alpha and beta fp32 in, o bf16
 # out; the states are added per sequence) and tensor-core flops of the chunked
@@ -355,6 +355,54 @@ def bench_decode(P, warmup, world, rank, dev):
                 steps=P.steps, bytes=state_b + io_b, state_bytes=state_b)
 
 
+# The time-split prefill: one 1M-token sequence with few heads (B=1, H=4,
+# T=2^20, d=128, bf16, the long workload's gates), where the plain sequential
+# walk keeps 2 H = 8 SMs busy.
+SPLIT_H, SPLIT_T = 4, 1 << 20
+
+
+def bench_timesplit(steps, warmup, world, rank, dev):
+    """kda_chunk_fwd_timesplit with the automatic segment count against the
+    same call without a split (segments = 1), whole calls timed."""
+    from gated_delta_rule_132_b200 import kda
+    P = I.LONG
+    x = I.make_prefill(1, SPLIT_T, SPLIT_H, P.d, P.dtype, P.gate_shift, 0.0,
+                       P.seed + 11 + 1000 * rank, device=f"cuda:{dev}")
+    L = kda.lib()
+    auto = None
+    for seg in range(2, 65):  # the count AUTO picks: the one whose workspace matches
+        if (L.kda_chunk_fwd_timesplit_workspace_size(1, SPLIT_T, SPLIT_H, P.d, P.d, 0, 1, seg) ==
+                L.kda_chunk_fwd_timesplit_workspace_size(1, SPLIT_T, SPLIT_H, P.d, P.d, 0, 1, 0)):
+            auto = seg
+            break
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, seg in (("sequential", 1), ("split", 0)):
+        ws = torch.empty(int(L.kda_chunk_fwd_timesplit_workspace_size(
+            1, SPLIT_T, SPLIT_H, P.d, P.d, 0, 1, seg)), dtype=torch.uint8, device=x["q"].device)
+        a = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, None, x["scale"])
+        for _ in range(warmup):
+            kda.kda_chunk_fwd_timesplit(*a, segments=seg, workspace=ws)
+        torch.cuda.synchronize()
+        barrier(world)
+
+        def step(i, ev):
+            ev[0].record(stream)
+            kda.kda_chunk_fwd_timesplit(*a, segments=seg, workspace=ws)
+            ev[1].record(stream)
+
+        total_ms, per = time_region(step, steps, stream, marks=2)
+        barrier(world)
+        ms = max_over_ranks(total_ms / steps, world)
+        out[name] = ms
+        del ws
+    chains = SPLIT_H
+    nseg = auto or 1
+    return dict(ms_seq=out["sequential"], ms_split=out["split"], segments=nseg,
+                tokens=SPLIT_T, ctas_seq=2 * chains,
+                ctas_pass1=chains * (2 + 4 * (nseg - 1)), ctas_pass2=chains * 2 * (nseg - 1))
+
+
 DECODE_TOKENS_T = 8  # tokens per multi-token decode call
 
 
@@ -501,6 +549,8 @@ def run_ours(args, world, rank, dev):
         dtok = None if args.no_decode else bench_decode_tokens(
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
         gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
+        tsp = None if args.no_timesplit else bench_timesplit(
+            min(args.steps, 5), args.warmup, world, rank, dev)
         bwd = None if args.no_backward else bench_backward(
             min(args.steps, 3), args.warmup, world, rank, dev, args.bwd_tokens)
     value = job_throughput(pre["tokens"], pre["ms"], world)
@@ -512,15 +562,19 @@ def run_ours(args, world, rank, dev):
     # own algorithmic bytes.
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     ach = pre["op_bytes"] / (kernels[dom]["ms"] / 1e3) / 1e9
-    traffic = {n: TRAFFIC_PER_RECORD[n] * pre["records"] for n in kernels}
+    traffic = {n: (TRAFFIC_PER_RECORD[n] * pre["records"] if TRAFFIC_PER_RECORD[n] else None)
+               for n in kernels}
+    known = all(v is not None for v in traffic.values())
     roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
             "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": traffic[dom],
             "peak_source": peak_kind,
             "bytes_per_launch": pre["op_bytes"], "ms_per_launch": round(kernels[dom]["ms"], 4),
             "note": "algorithmic bytes of the whole prefill / the dominant kernel's time",
             "traffic_vs_algorithmic": {
-                dom: round(traffic[dom] / kernels[dom]["bytes"], 3),
-                "prefill": round(sum(traffic.values()) / pre["op_bytes"], 3)},
+                dom: (round(traffic[dom] / kernels[dom]["bytes"], 3)
+                      if traffic[dom] is not None else None),
+                "prefill": (round(sum(traffic.values()) / pre["op_bytes"], 3)
+                            if known else None)},
             "traffic_note": "ncu DRAM bytes per record on the chunked workload x records"}
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -582,8 +636,23 @@ def run_ours(args, world, rank, dev):
             "kernels_ms": {"prepare": round(gdn["prep_ms"], 4), "carry": round(gdn["carry_ms"], 4)},
             "op_roofline": {"bound": "hbm", "achieved": round(g_ach, 1), "peak": hbm,
                             "unit": "GB/s", "frac": round(g_ach / hbm, 4),
-                            "traffic": TRAFFIC_PER_RECORD["gdn_prepare"] * pre["records"],
+                            "traffic": (TRAFFIC_PER_RECORD["gdn_prepare"] * pre["records"]
+                                        if TRAFFIC_PER_RECORD["gdn_prepare"] else None),
                             "bytes_per_step": gdn["in_bytes"] + pre["out_bytes"]}}
+    if tsp is not None:
+        line["timesplit"] = {
+            "workload": f"long_bf16_B1_H{SPLIT_H}_T{SPLIT_T}_d128",
+            "value": round(job_throughput(tsp["tokens"], tsp["ms_split"], world), 1),
+            "unit": "tokens/s", "ms_per_step": round(tsp["ms_split"], 4),
+            "segments": tsp["segments"],
+            "sequential": {"value": round(job_throughput(tsp["tokens"], tsp["ms_seq"], world), 1),
+                           "ms_per_step": round(tsp["ms_seq"], 4),
+                           "sms_busy_in_walk": tsp["ctas_seq"]},
+            "sms_busy_in_walk": {"pass1": min(148, tsp["ctas_pass1"]),
+                                 "pass2": min(148, tsp["ctas_pass2"])},
+            "speedup": round(tsp["ms_seq"] / tsp["ms_split"], 3),
+            "note": "whole kda_chunk_fwd_timesplit calls (prep + walk); one CTA per SM in the "
+                    "sequential walk"}
     if bwd is not None:
         tf = bwd["token_heads"] * BWD_FLOP_PER_TOKEN_HEAD / (bwd["kern_ms"] / 1e3) / 1e12
         line["backward"] = {
@@ -666,6 +735,8 @@ def main():
                     help="skip the backward (kda_chunk_bwd) measurement")
     ap.add_argument("--bwd-tokens", type=int, default=BWD_T,
                     help="tokens of the backward measurement (all 32 heads)")
+    ap.add_argument("--no-timesplit", action="store_true",
+                    help="skip the time-split prefill measurement (B=1, H=4, T=2^20)")
     ap.add_argument("--no-gdn", action="store_true",
                     help="skip the one-gate-per-head (GDN) variant of the prefill")
     ap.add_argument("--e2e-steps", type=int, default=10)

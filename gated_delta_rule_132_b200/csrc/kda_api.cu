@@ -51,6 +51,7 @@ kda_status_t describe(int B, int T, int H, int dk, int dv, int n_seqs, bool varl
     p->total_tokens = total;
     p->max_chunks = (int)chunks;
     p->gate_per_channel = 1;
+    p->nseg = 1;
     return KDA_OK;
 }
 
@@ -59,8 +60,31 @@ bool use_tc(const kda::Problem &p, int algo) {
     return kda::tc_supported(p);
 }
 
-size_t required_bytes(const kda::Problem &p, bool tc) {
-    return tc ? kda::tc_workspace_layout(p).total : kda::simt_workspace_layout(p).total;
+bool tc_only(int algo) { return algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT; }
+
+// Algorithm values beyond the public kda_algo_t: the tensor-core path with an
+// explicit number of time segments (kda_chunk_fwd_timesplit).
+constexpr int kAlgoSegmentsBase = 1000;
+
+bool algo_ok(int algo)
+{
+    return algo == KDA_ALGO_AUTO || algo == KDA_ALGO_SIMT || algo == KDA_ALGO_TCGEN05 ||
+           algo == KDA_ALGO_TCGEN05_SEQUENTIAL ||
+           (algo > kAlgoSegmentsBase && algo <= kAlgoSegmentsBase + kda::kMaxSegments);
+}
+
+// Time segments of the sequential phase on the tensor-core path for `algo`.
+int segments_for(const kda::Problem &p, int algo)
+{
+    if (algo == KDA_ALGO_TCGEN05_SEQUENTIAL) return 1;
+    if (algo > kAlgoSegmentsBase) return algo - kAlgoSegmentsBase;
+    return kda::tc_auto_segments(p);
+}
+
+size_t required_bytes(kda::Problem &p, bool tc, int algo) {
+    if (!tc) return kda::simt_workspace_layout(p).total;
+    p.nseg = segments_for(p, algo);
+    return kda::tc_workspace_layout(p).total;
 }
 
 }  // namespace
@@ -122,13 +146,21 @@ int kda_version(void) { return 300; }  // 0.3.0: device status word, launch coun
 size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
                                        kda_dtype_t dt, int algo)
 {
-    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TCGEN05) return 0;
+    if (!algo_ok(algo)) return 0;
     kda::Problem p;
     const bool varlen = n_seqs > 0 && B == 1;
     if (describe(B, T, H, dk, dv, n_seqs, varlen, dt, &p) != KDA_OK) return 0;
     const bool tc = use_tc(p, algo);
-    if (algo == KDA_ALGO_TCGEN05 && !tc) return 0;
-    return required_bytes(p, tc);
+    if (tc_only(algo) && !tc) return 0;
+    return required_bytes(p, tc, algo);
+}
+
+size_t kda_chunk_fwd_timesplit_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                              kda_dtype_t dt, int segments)
+{
+    if (segments < 0 || segments > kda::kMaxSegments) return 0;
+    return kda_chunk_fwd_workspace_size_ex(
+        B, T, H, dk, dv, n_seqs, dt, segments == 0 ? KDA_ALGO_TCGEN05 : kAlgoSegmentsBase + segments);
 }
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
@@ -147,8 +179,7 @@ static kda_status_t chunk_fwd_phases(const void *q, const void *k, const void *v
                                      float *S_final, void *workspace, size_t workspace_bytes,
                                      int algo, int phases, int gate_per_channel, void *stream)
 {
-    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TCGEN05)
-        return KDA_ERR_INVALID_ARG;
+    if (!algo_ok(algo)) return KDA_ERR_INVALID_ARG;
     kda::Problem p;
     kda_status_t st = describe(B, T, H, dk, dv, n_seqs, cu_seqlens != nullptr, dt, &p);
     if (st != KDA_OK) return st;
@@ -160,8 +191,8 @@ static kda_status_t chunk_fwd_phases(const void *q, const void *k, const void *v
         if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
     if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_ALIGNMENT;
     const bool tc = use_tc(p, algo);
-    if (algo == KDA_ALGO_TCGEN05 && !tc) return KDA_ERR_UNSUPPORTED;
-    const size_t need = required_bytes(p, tc);
+    if (tc_only(algo) && !tc) return KDA_ERR_UNSUPPORTED;
+    const size_t need = required_bytes(p, tc, algo);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
 
     p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.S0 = S0;
@@ -229,6 +260,18 @@ kda_status_t kda_chunk_fwd_carry(const void *q, const void *k, const void *v, kd
                                  void *workspace, size_t workspace_bytes, int algo, void *stream)
 {
     return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseCarry, 1, stream);
+}
+
+kda_status_t kda_chunk_fwd_timesplit(const void *q, const void *k, const void *v,
+                                     kda_dtype_t dt, const float *log_alpha, const float *beta,
+                                     const float *S0, const int32_t *cu_seqlens, int n_seqs,
+                                     int B, int T, int H, int dk, int dv, float scale, void *o,
+                                     float *S_final, void *workspace, size_t workspace_bytes,
+                                     int segments, void *stream)
+{
+    if (segments < 0 || segments > kda::kMaxSegments) return KDA_ERR_INVALID_ARG;
+    const int algo = segments == 0 ? KDA_ALGO_TCGEN05 : kAlgoSegmentsBase + segments;
+    return chunk_fwd_phases(KDA_CHUNK_ARGS, algo, kda::kPhaseAll, 1, stream);
 }
 
 kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtype_t dt,

@@ -15,11 +15,11 @@
 // shared memory, and stream the updated rows back. Loads and stores use the
 // evict-first cache hint: the state is touched once per call.
 //
-// The same kernel applies T consecutive tokens per (sequence, head) with the
-// state kept in registers between them (multi-token decode, or continuing a
-// prefill by a few tokens): the state still crosses HBM once each way, and
-// each token costs three CTA barriers and its own few hundred bytes, with the
-// next token's vectors loaded while the current one is reduced.
+// Several consecutive tokens per (sequence, head) (multi-token decode, or
+// continuing a prefill by a few tokens) run in decode_tokens_kernel with the
+// state kept in registers between them: the state still crosses HBM once each
+// way, the tokens' vectors are staged in shared memory ahead of use, and each
+// token costs two CTA barriers and its own few hundred bytes.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -127,12 +127,198 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     }
 }
 
+// Several tokens per call (T >= 2). The state stays in registers as in
+// decode_kernel; the tokens' vectors are staged in shared memory in blocks of
+// kTokBlock tokens with cp.async, two blocks in flight, so a token never waits
+// for a global load. When a block lands, its log-decays become decays
+// (alpha = exp(log_alpha)) and each warp forms one token's k^T q. Per token:
+// partial S'^T k and S'^T q -> barrier -> u and o per value column -> barrier
+// -> S += k u^T. The reduction and u buffers alternate between tokens, so those
+// two barriers are the only ones a token needs.
+constexpr int kTokBlock = 8;
+
+template <int DK, int DV, typename TIn>
+struct TokSmem {
+    static constexpr int CG = DV / 4, RG = kDecodeThreads / CG;
+    // one block of staged tokens
+    static constexpr size_t kLa = 0;                                         // fp32 [TB][DK] (alpha after landing)
+    static constexpr size_t kK = kLa + sizeof(float) * kTokBlock * DK;        // TIn [TB][DK]
+    static constexpr size_t kQ = kK + sizeof(TIn) * kTokBlock * DK;          // TIn [TB][DK]
+    static constexpr size_t kV = kQ + sizeof(TIn) * kTokBlock * DK;          // TIn [TB][DV]
+    static constexpr size_t kB = kV + sizeof(TIn) * kTokBlock * DV;          // fp32 [TB] beta
+    static constexpr size_t kKq = kB + sizeof(float) * kTokBlock;            // fp32 [TB] k^T q
+    static constexpr size_t kBlock = (kKq + sizeof(float) * kTokBlock + 15) / 16 * 16;
+    static constexpr size_t kRed = 2 * kBlock;                               // fp32 [2][2][RG][DV]
+    static constexpr size_t kU = kRed + sizeof(float) * 2 * 2 * RG * DV;     // fp32 [2][DV]
+    static constexpr size_t kBytes = kU + sizeof(float) * 2 * DV;
+};
+
+template <int DK, int DV, typename TIn>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+decode_tokens_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
+                     const TIn *__restrict__ v, const float *__restrict__ log_alpha,
+                     const float *__restrict__ beta, float *__restrict__ S, int T, int H,
+                     int gate_per_channel, float scale, TIn *__restrict__ o)
+{
+    using L = TokSmem<DK, DV, TIn>;
+    constexpr int CG = L::CG, RG = L::RG, RPT = DK / RG;
+    static_assert(DK % RG == 0 && RPT >= 1, "unsupported head size");
+    static_assert(DV <= kDecodeThreads, "one value column per thread");
+    extern __shared__ __align__(16) uint8_t smem[];
+
+    const int unit = blockIdx.x;  // n * H + h
+    const int n = unit / H, h = unit - n * H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cg = tid % CG, rg = tid / CG;
+    float *Su = S + (size_t)unit * DK * DV;
+
+    float4 st[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+        st[r] = __ldcs(reinterpret_cast<const float4 *>(Su + (size_t)(r * RG + rg) * DV) + cg);
+
+    const int nblocks = (T + kTokBlock - 1) / kTokBlock;
+    auto tok_index = [&](int t) { return ((size_t)n * T + t) * H + h; };  // (n, t, h)
+    // Stage block b (tokens kTokBlock b ..) into buffer b & 1, as one cp.async group.
+    auto stage = [&](int b) {
+        uint8_t *buf = smem + (size_t)(b & 1) * L::kBlock;
+        const int t0 = b * kTokBlock, nt = min(kTokBlock, T - t0);
+        constexpr int kLaG = DK * 4 / 16, kKG = DK * (int)sizeof(TIn) / 16, kVG = DV * (int)sizeof(TIn) / 16;
+        constexpr int kPer = kLaG + 2 * kKG + kVG;  // 16-byte granules per token
+        for (int g = tid; g < nt * kPer; g += kDecodeThreads) {
+            const int tt = g / kPer, r = g % kPer;
+            const size_t tok = tok_index(t0 + tt);
+            const void *src;
+            uint8_t *dst;
+            if (r < kLaG) {
+                if (!gate_per_channel) continue;
+                src = log_alpha + tok * DK + 4 * r;
+                dst = buf + L::kLa + ((size_t)tt * DK + 4 * r) * 4;
+            } else if (r < kLaG + kKG) {
+                const int e = (r - kLaG) * (16 / (int)sizeof(TIn));
+                src = k + tok * DK + e;
+                dst = buf + L::kK + ((size_t)tt * DK + e) * sizeof(TIn);
+            } else if (r < kLaG + 2 * kKG) {
+                const int e = (r - kLaG - kKG) * (16 / (int)sizeof(TIn));
+                src = q + tok * DK + e;
+                dst = buf + L::kQ + ((size_t)tt * DK + e) * sizeof(TIn);
+            } else {
+                const int e = (r - kLaG - 2 * kKG) * (16 / (int)sizeof(TIn));
+                src = v + tok * DV + e;
+                dst = buf + L::kV + ((size_t)tt * DV + e) * sizeof(TIn);
+            }
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                         ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+        }
+        if (tid < nt) {  // beta, and the scalar gate of one-gate-per-head calls
+            const size_t tok = tok_index(t0 + tid);
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                         ::"r"((uint32_t)__cvta_generic_to_shared(buf + L::kB + 4 * tid)),
+                           "l"(beta + tok) : "memory");
+            if (!gate_per_channel)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                             ::"r"((uint32_t)__cvta_generic_to_shared(buf + L::kLa + 4 * tid * DK)),
+                               "l"(log_alpha + tok) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    stage(0);
+    if (nblocks > 1) stage(1);
+
+    float *red = reinterpret_cast<float *>(smem + L::kRed);  // [2][2][RG][DV]
+    float *su = reinterpret_cast<float *>(smem + L::kU);     // [2][DV]
+    for (int b = 0; b < nblocks; ++b) {
+        uint8_t *buf = smem + (size_t)(b & 1) * L::kBlock;
+        const int t0 = b * kTokBlock, nt = min(kTokBlock, T - t0);
+        // this block's copies (the later block's may stay in flight)
+        if (b + 1 < nblocks) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        float *sa = reinterpret_cast<float *>(buf + L::kLa);
+        const TIn *sk = reinterpret_cast<const TIn *>(buf + L::kK);
+        const TIn *sq = reinterpret_cast<const TIn *>(buf + L::kQ);
+        const TIn *sv = reinterpret_cast<const TIn *>(buf + L::kV);
+        const float *sb = reinterpret_cast<const float *>(buf + L::kB);
+        float *skq = reinterpret_cast<float *>(buf + L::kKq);
+        // decays and k^T q of the block's tokens
+        if (gate_per_channel) {
+            for (int e = tid; e < nt * DK; e += kDecodeThreads) sa[e] = expf(sa[e]);
+        } else if (tid < nt) {
+            const float a = expf(sa[tid * DK]);
+            for (int i = 0; i < DK; ++i) sa[tid * DK + i] = a;
+        }
+        if (warp < nt) {
+            float acc = 0.f;
+            for (int i = lane; i < DK; i += 32) acc += to_f32(sk[warp * DK + i]) * to_f32(sq[warp * DK + i]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) skq[warp] = acc;
+        }
+        __syncthreads();
+        for (int tt = 0; tt < nt; ++tt) {
+            const int t = t0 + tt, par = t & 1;
+            const float *al = sa + tt * DK;
+            const TIn *kt = sk + tt * DK;
+            const TIn *qt = sq + tt * DK;
+            // S' = Diag(alpha) S and this thread's partial S'^T k, S'^T q
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), bq = a;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const int i = r * RG + rg;
+                const float ali = al[i], ki = to_f32(kt[i]), qi = to_f32(qt[i]);
+                st[r].x *= ali; st[r].y *= ali; st[r].z *= ali; st[r].w *= ali;
+                a.x += st[r].x * ki; a.y += st[r].y * ki; a.z += st[r].z * ki; a.w += st[r].w * ki;
+                bq.x += st[r].x * qi; bq.y += st[r].y * qi; bq.z += st[r].z * qi; bq.w += st[r].w * qi;
+            }
+            float *rk = red + ((size_t)par * 2 + 0) * RG * DV, *rq = red + ((size_t)par * 2 + 1) * RG * DV;
+            reinterpret_cast<float4 *>(rk + rg * DV)[cg] = a;
+            reinterpret_cast<float4 *>(rq + rg * DV)[cg] = bq;
+            __syncthreads();
+            // u = beta (v - S'^T k), o = scale (S'^T q + (k^T q) u), per value column
+            if (tid < DV) {
+                float sk2 = 0.f, sq2 = 0.f;
+#pragma unroll
+                for (int g = 0; g < RG; ++g) { sk2 += rk[g * DV + tid]; sq2 += rq[g * DV + tid]; }
+                const float u = sb[tt] * (to_f32(sv[tt * DV + tid]) - sk2);
+                su[par * DV + tid] = u;
+                o[tok_index(t) * DV + tid] = from_f32<TIn>(scale * (sq2 + skq[tt] * u));
+            }
+            __syncthreads();
+            // S = S' + k u^T
+            const float4 u4 = reinterpret_cast<const float4 *>(su + par * DV)[cg];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const float ki = to_f32(kt[r * RG + rg]);
+                st[r].x += ki * u4.x; st[r].y += ki * u4.y; st[r].z += ki * u4.z; st[r].w += ki * u4.w;
+            }
+        }
+        // every thread is done with this buffer before block b + 2 lands in it
+        __syncthreads();
+        if (b + 2 < nblocks) stage(b + 2);
+    }
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+        __stcs(reinterpret_cast<float4 *>(Su + (size_t)(r * RG + rg) * DV) + cg, st[r]);
+}
+
 template <int D, typename TIn>
 cudaError_t launch_d(const void *q, const void *k, const void *v, const float *la,
                      const float *beta, float *S, int units, int T, int H, int gpc, float scale,
                      void *o, cudaStream_t st)
 {
-    decode_kernel<D, D, TIn><<<units, kDecodeThreads, 0, st>>>(
+    if (T == 1) {
+        decode_kernel<D, D, TIn><<<units, kDecodeThreads, 0, st>>>(
+            static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v),
+            la, beta, S, T, H, gpc, scale, static_cast<TIn *>(o));
+        note_launch();
+        return cudaGetLastError();
+    }
+    using L = TokSmem<D, D, TIn>;
+    auto kern = decode_tokens_kernel<D, D, TIn>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::kBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<units, kDecodeThreads, L::kBytes, st>>>(
         static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v),
         la, beta, S, T, H, gpc, scale, static_cast<TIn *>(o));
     note_launch();

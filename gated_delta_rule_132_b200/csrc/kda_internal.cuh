@@ -38,7 +38,11 @@ struct Problem {
     long long total_tokens;     // B * T (packed time axis length)
     int max_chunks;             // upper bound on chunks over all sequences
     int gate_per_channel;       // 1: log_alpha [.., H, dk] (KDA); 0: [.., H] (one gate per head)
+    int nseg;                   // tensor-core path: time segments of the sequential phase (1: none)
 };
+
+// Most time segments the tensor-core path splits a sequence into.
+constexpr int kMaxSegments = 64;
 
 // Sequence plan in the workspace: for n in [0, N], the sanitised packed start
 // token seq_start[n] and first global chunk chunk_off[n] (both int32; entry N
@@ -100,6 +104,8 @@ cudaError_t launch_simt_prefill(const Problem &p, void *workspace, int phases,
 cudaError_t launch_tc_prefill(const Problem &p, void *workspace, int phases,
                               cudaStream_t stream);
 bool tc_supported(const Problem &p);
+// Time segments the tensor-core path uses for this problem when left to choose.
+int tc_auto_segments(const Problem &p);
 // Backward of the prefill (fp32 CUDA cores): gradients of <dO, o> + <dS_final, S_final>.
 WorkspaceLayout bwd_workspace_layout(const Problem &p);
 cudaError_t launch_backward(const Problem &p, const void *dO, const float *dS_final,

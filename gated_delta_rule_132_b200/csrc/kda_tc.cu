@@ -43,39 +43,39 @@ constexpr int kSlice = 64;  // value columns per carry CTA
 constexpr int kSlices = D / kSlice;
 
 // Workspace record per (chunk, head), bytes. Every piece is a verbatim image of
-// a shared-memory operand so the carry kernel can bulk-copy it.
+// a shared-memory operand of the carry kernel, which bulk-copies it. The carry
+// needs one group of MMAs per chunk (see the carry below):
+//     D = [S^T | U~^T] . [[-N, Q']^T ; [K^, P^T]]   (N = K^^T W, Q' = Q~ - P W)
+// so the record holds the B operand of that group in two K ranges (keys, then
+// tokens), each as 192 K-major rows: 128 state rows (one per key channel) and
+// 64 output rows (one per token).
 struct Record {
-    static constexpr uint32_t kA1 = 0;        // [W; Q~] 128x128 bf16, K-major, SW128, 2 K-blocks
-    static constexpr uint32_t kKh = 32768;    // K^^T 128x64 bf16, MN-major, SW128, 2 MN-blocks
-    static constexpr uint32_t kP = 49152;     // P 64x64 bf16, K-major, SW128
-    static constexpr uint32_t kG = 57344;     // gamma fp32 [128]
-    static constexpr uint32_t kU = 57856;     // U~^T fp32 [2 halves][64 value cols][64 tokens], 16B-chunk swizzled
+    static constexpr uint32_t kBk = 0;        // [2 key blocks][192 rows][128 B] bf16 K-major SW128:
+                                              //   rows 0..127: -N[i][i'], rows 128..191: Q'[t][i]
+    static constexpr uint32_t kBt = 49152;    // [192 rows][128 B] bf16 K-major SW128:
+                                              //   rows 0..127: K^[t][i] (row i), rows 128..191: P[t][s]
+    static constexpr uint32_t kU = 73728;     // U~^T bf16 [2 halves][64 value cols][128 B] K-major SW128
+    static constexpr uint32_t kG = 90112;     // gamma fp32 [128]
     static constexpr uint32_t kBytes = 90624;
+    static constexpr uint32_t kBlk = 24576;   // one 192-row block
+    static constexpr uint32_t kOut = 16384;   // rows 128..191 start 16 KB into a block
 };
-static_assert(Record::kU + kSlices * C * kSlice * 4 == Record::kBytes, "record size");
+static_assert(Record::kG + 512 == Record::kBytes, "record size");
 
 // Shared-memory layout of the carry kernel (offsets from a 1024-aligned base).
 struct CarrySmem {
-    static constexpr uint32_t kA1 = 0;         // 32768: [W; Q~], B of MMA1 (K-major)
-    static constexpr uint32_t kKh = 32768;     // 16384: K^, B of MMA2 (MN-major)
-    static constexpr uint32_t kP = 49152;      // 8192:  P, B of MMA3 (K-major)
-    static constexpr uint32_t kU = 57344;      // 16384: U~^T of this half, fp32
-    static constexpr uint32_t kG = 73728;      // 512:   gamma
-    static constexpr uint32_t kStage = 74752;  // stage stride (1024-aligned)
-    static constexpr uint32_t kSt = 2 * kStage;        // S^T bf16 64x128, A of MMA1 (K-major, 2 K-blocks)
-    static constexpr uint32_t kUt = kSt + 16384;       // U^T bf16 64x64, A of MMA2/MMA3 (K-major)
-    static constexpr uint32_t kOs = kUt + 8192;        // output staging, 1 KB per state warp
+    static constexpr uint32_t kBk = 0;         // 49152: B over the keys (K-major, 2 K-blocks)
+    static constexpr uint32_t kBt = 49152;     // 24576: B over the tokens (K-major)
+    static constexpr uint32_t kU = 73728;      // 8192:  U~^T of this half, A over the tokens
+    static constexpr uint32_t kG = 81920;      // 512:   gamma
+    static constexpr uint32_t kStage = 82944;  // stage stride (1024-aligned)
+    static constexpr uint32_t kSt = 2 * kStage;        // 2 x S^T bf16 64x128, A over the keys (K-major, 2 K-blocks)
+    static constexpr uint32_t kOs = kSt + 2 * 16384;   // output staging, 1 KB per state warp
     static constexpr uint32_t kBar = kOs + 8192;       // mbarriers
     static constexpr uint32_t kBytes = kBar + 256 + 1024;  // + alignment slack
 };
-static_assert(CarrySmem::kSt % 1024 == 0 && CarrySmem::kUt % 1024 == 0, "operand alignment");
-
-__device__ __forceinline__ uint32_t u_swz(uint32_t r, uint32_t jj)
-{
-    // byte offset of element [r][jj] of a 64x64 fp32 tile (rows of 256 bytes):
-    // 16-byte chunks XORed by row
-    return r * 256u + ((((jj >> 2) ^ (r & 15u)) << 4) | ((jj & 3u) << 2));
-}
+static_assert(CarrySmem::kSt % 1024 == 0 && CarrySmem::kStage % 1024 == 0, "operand alignment");
+static_assert(CarrySmem::kBytes <= 227 * 1024, "carry shared memory");
 
 struct TcParams {
     const __nv_bfloat16 *q, *k, *v;
@@ -90,6 +90,13 @@ struct TcParams {
     int *fix_count;    // number of chunks listed for the exact fixup
     uint32_t spin;     // poll limit of every bounded wait
     int starve;        // debugging: the carry's producer issues no copies
+    // time split of the sequential phase (see the carry kernel): segments per
+    // sequence, the launch's pass, and the segment states
+    // [3 kinds][nseg][N][H][D][D] fp32 (kind 0: state from a zero start,
+    // 1: transition, 2: state at the segment's end)
+    int nseg;
+    int pass;          // 0: no split, 1: first pass, 2: second pass
+    float *seg;
     int *fix_list;     // chunk * H + head, one per listed chunk
     // q, k, v and log_alpha as 3-D tensors {channel, head, token} for TMA tile
     // loads of 128 bytes of channels x 1 head x 64 tokens in the 128-byte
@@ -115,16 +122,24 @@ __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int c)
 // its factorised exponentials (a decay of more than 80 nats inside half a
 // chunk); for ordinary gates the list is empty and the kernel exits at once.
 constexpr int kPrepThreads = 256;
+constexpr int DP = D + 1;  // padded fp32 row of the fixup's [C][D] arrays
+
+// bf16 element (row, k) of a K-major SW128 block whose rows are 128 bytes
+__device__ __forceinline__ __nv_bfloat16 *kmaj(uint8_t *block, int row, int k)
+{
+    return reinterpret_cast<__nv_bfloat16 *>(block + tc::sw128((uint32_t)row, 2u * (uint32_t)k));
+}
 
 __device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
 {
-    constexpr int DP = D + 1;
-    float *sk = smem;               // [C][DP]
-    float *sq = sk + C * DP;        // [C][DP]
-    float *sg = sq + C * DP;        // [C][DP]
-    float *sv = sg + C * DP;        // [C][D]
+    float *sk = smem;               // [C][DP]  k, then beta e^g k, then W
+    float *sq = sk + C * DP;        // [C][DP]  q, then Q~
+    float *sg = sq + C * DP;        // [C][DP]  cumulative log-decay g
+    float *skh = sg + C * DP;       // [C][DP]  K^
+    float *sv = skh + C * DP;       // [C][D]   v, then beta v, then U~
     float *sA = sv + C * D;         // [C][C+1]
-    float *sb = sA + C * (C + 1);   // [C]
+    float *sP = sA + C * (C + 1);   // [C][C+1]
+    float *sb = sP + C * (C + 1);   // [C]
 
     const int H = p.H;
     const int n = find_seq(p.chunk_off, p.N, c);
@@ -153,12 +168,6 @@ __device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
     __syncthreads();
 
     uint8_t *rec = p.rec + ((size_t)c * H + h) * Record::kBytes;
-    __nv_bfloat16 *a1 = reinterpret_cast<__nv_bfloat16 *>(rec + Record::kA1);
-    __nv_bfloat16 *kh = reinterpret_cast<__nv_bfloat16 *>(rec + Record::kKh);
-    __nv_bfloat16 *pp = reinterpret_cast<__nv_bfloat16 *>(rec + Record::kP);
-    float *gg = reinterpret_cast<float *>(rec + Record::kG);
-    uint8_t *uu = rec + Record::kU;
-
     const int warp = tid >> 5, lane = tid & 31;
     for (int r = warp; r < C; r += kPrepThreads / 32) {
         for (int s = lane; s < C; s += 32) {
@@ -172,27 +181,23 @@ __device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
                 }
             }
             sA[r * (C + 1) + s] = (s < r) ? sb[r] * akk : 0.f;
-            pp[tc::sw128(r, 2 * s) / 2] = __float2bfloat16_rn(pqk);
+            sP[r * (C + 1) + s] = (s <= r) ? pqk : 0.f;
         }
     }
-    // Q~ (rows 64..127 of A1), K^ (MN-major image) and gamma.
+    __syncthreads();
+    // Q~ in place, K^, gamma; then the solve's right-hand sides
     for (int idx = tid; idx < C * D; idx += kPrepThreads) {
         const int r = idx / D, i = idx % D;
         const float g = sg[r * DP + i], gC = sg[(C - 1) * DP + i];
-        const uint32_t kb = (uint32_t)(i >> 6) * 16384u;
-        a1[(kb + tc::sw128(64 + r, 2 * (i & 63))) / 2] = __float2bfloat16_rn(expf(g) * sq[r * DP + i]);
-        kh[((uint32_t)(i >> 6) * 8192u + tc::sw128(r, 2 * (i & 63))) / 2] =
-            __float2bfloat16_rn(expf(gC - g) * sk[r * DP + i]);
-    }
-    for (int i = tid; i < D; i += kPrepThreads) gg[i] = expf(sg[(C - 1) * DP + i]);
-    __syncthreads();
-    for (int idx = tid; idx < C * D; idx += kPrepThreads) {
-        const int r = idx / D, i = idx % D;
-        sk[r * DP + i] *= sb[r] * expf(sg[r * DP + i]);
+        sq[r * DP + i] *= expf(g);
+        skh[r * DP + i] = expf(gC - g) * sk[r * DP + i];
+        sk[r * DP + i] *= sb[r] * expf(g);
         sv[r * D + i] *= sb[r];
     }
+    for (int i = tid; i < D; i += kPrepThreads)
+        reinterpret_cast<float *>(rec + Record::kG)[i] = expf(sg[(C - 1) * DP + i]);
     __syncthreads();
-    for (int col = tid; col < 2 * D; col += kPrepThreads) {
+    for (int col = tid; col < 2 * D; col += kPrepThreads) {  // W and U~ by forward substitution
         float *x = col < D ? sk + col : sv + (col - D);
         const int stride = col < D ? DP : D;
         for (int r = 1; r < C; ++r) {
@@ -202,12 +207,28 @@ __device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
         }
     }
     __syncthreads();
+    // -N = -K^^T W (rows i of the key block i'/64), Q' = Q~ - P W (rows 128 + t)
+    for (int idx = tid; idx < D * D; idx += kPrepThreads) {
+        const int i = idx / D, i2 = idx % D;
+        float acc = 0.f;
+        for (int t = 0; t < C; ++t) acc += skh[t * DP + i] * sk[t * DP + i2];
+        *kmaj(rec + Record::kBk + (i2 >> 6) * Record::kBlk, i, i2 & 63) = __float2bfloat16_rn(-acc);
+    }
     for (int idx = tid; idx < C * D; idx += kPrepThreads) {
-        const int r = idx / D, i = idx % D;
-        const uint32_t kb = (uint32_t)(i >> 6) * 16384u;
-        a1[(kb + tc::sw128(r, 2 * (i & 63))) / 2] = __float2bfloat16_rn(sk[r * DP + i]);
-        const int half = i >> 6, jj = i & 63;
-        *reinterpret_cast<float *>(uu + half * 16384 + u_swz(jj, r)) = sv[r * D + i];
+        const int t = idx / D, i2 = idx % D;
+        float acc = sq[t * DP + i2];
+        for (int s2 = 0; s2 <= t; ++s2) acc -= sP[t * (C + 1) + s2] * sk[s2 * DP + i2];
+        *kmaj(rec + Record::kBk + (i2 >> 6) * Record::kBlk, 128 + t, i2 & 63) = __float2bfloat16_rn(acc);
+    }
+    // K^ as rows i over the tokens, P as rows 128 + t, U~^T as rows j of its half
+    for (int idx = tid; idx < D * C; idx += kPrepThreads) {
+        const int i = idx / C, t = idx % C;
+        *kmaj(rec + Record::kBt, i, t) = __float2bfloat16_rn(skh[t * DP + i]);
+        *kmaj(rec + Record::kU + (i >> 6) * 8192, i & 63, t) = __float2bfloat16_rn(sv[t * D + i]);
+    }
+    for (int idx = tid; idx < C * C; idx += kPrepThreads) {
+        const int t = idx / C, s2 = idx % C;
+        *kmaj(rec + Record::kBt, 128 + t, s2) = __float2bfloat16_rn(sP[t * (C + 1) + s2]);
     }
     __syncthreads();  // the caller reuses shared memory for its next chunk
 }
@@ -246,6 +267,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams
 //  5. Everything goes to the record in the carry kernel's operand layouts.
 constexpr int kPrep2Threads = 256;
 
+constexpr uint32_t kLdBytes = 68 * 4;  // one row of the fp32 A / T matrices (kLd floats)
+
 struct Prep2Smem {
     static constexpr uint32_t kAop = 0;        // 32768: [kb][128 rows][128B]
     static constexpr uint32_t kA = 0;          // fp32 A [64][kLd], after MMA-AP
@@ -261,7 +284,17 @@ struct Prep2Smem {
     static constexpr uint32_t kB = 106496;     // 256:   beta [64]
     static constexpr uint32_t kBar = 106752;   // barriers + tmem slot + flags
     static constexpr uint32_t kBytes = kBar + 64 + 1024;
+    // Later tenants of the same memory (each region is dead by then):
+    static constexpr uint32_t kKhT = 0;        // 16384: K^ as rows i over the tokens, after the inverse
+    static constexpr uint32_t kP = 18432;      // 8192:  P (K-major rows t), from the A/P read-out on
+    static constexpr uint32_t kW = 32768;      // 16384: W bf16 MN-major image, after MMA-WU
+    static constexpr uint32_t kQp = 32768;     // 16384: Q' staging (2 key blocks of 8 KB), after MMA-NP
+    static constexpr uint32_t kN0 = 57344;     // 16384: -N staging, key block 0, after MMA-WU
+    static constexpr uint32_t kUs = 73728;     // 16384: U~^T bf16 staging, after MMA-WU
+    static constexpr uint32_t kN1 = 90112;     // 16384: -N staging, key block 1, after MMA-WU
 };
+static_assert(Prep2Smem::kP >= 64 * kLdBytes && Prep2Smem::kP + 8192 <= Prep2Smem::kBop,
+              "P lives between the fp32 A matrix and the B operand");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 {
@@ -467,6 +500,148 @@ __device__ __forceinline__ void invert_unit_lower64_by_distance(const float *As,
     __syncthreads();
 }
 
+// Where finish_record keeps its operands and staging (offsets from the
+// 1024-aligned shared-memory base; each region must be dead when it is used).
+struct FinishSmem {
+    uint32_t w;     // 16384: W bf16 MN-major image (B of MMA-NP)
+    uint32_t us;    // 16384: U~^T bf16 staging
+    uint32_t kht;   // 16384: K^ rows i over the tokens (A of MMA-NP), already in place
+    uint32_t pp;    // 8192:  P rows t (A of MMA-NP), already in place
+    uint32_t n0;    // 16384: -N staging, key block 0 (after MMA-NP)
+    uint32_t n1;    // 16384: -N staging, key block 1 (after MMA-NP)
+    uint32_t qp;    // 16384: Q' staging (2 key blocks of 8 KB, after MMA-NP)
+};
+
+// The end of both prep kernels, once the W and U~^T MMAs (TMEM columns 0..127
+// lanes 0..63, and columns 128..191 lanes 0..127) are committed to bar_wu and K^
+// and P are in shared memory:
+//   1. W -> bf16 MN-major image; U~^T -> bf16 rows j of its half, sent to the record;
+//   2. MMA-NP: N = K^^T W (M = 128, columns 0..127) and P W (M = 64, columns 128..255);
+//   3. -N and Q' = Q~ - P W (Q~ from qt(t, key block, chunk) as 8 floats) as record
+//      images, sent with bulk stores; then every copy and MMA is drained.
+// Ends with the CTA's asynchronous work finished (TMEM may be released).
+template <typename QtFn>
+__device__ __forceinline__ void finish_record(uint8_t *sm, const FinishSmem &f, uint32_t tmem,
+                                              uint8_t *rec, uint64_t *bar_wu, uint64_t *bar_np,
+                                              uint64_t *bar_ld, uint64_t *bar_fin,
+                                              volatile int *abort, const TcParams &p, int code,
+                                              QtFn qt)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lg = warp & 3, wh = warp >> 2;
+    const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
+    {
+        tc::mbar_wait(bar_wu, 0, abort, p.err, code, p.spin);
+        tc::tc_fence_after_sync();
+        const int row = lg * 32 + lane;
+        float w[32];
+        if (lg < 2) {  // W: lanes 0..63 are the tokens
+            uint8_t *wb = sm + f.w + (uint32_t)wh * 8192;
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
+                    *reinterpret_cast<uint4 *>(wb + tc::sw128(row, (q2 * 4 + c16) * 16)) =
+                        make_uint4(u[0], u[1], u[2], u[3]);
+                }
+            }
+        }
+        // U~^T: lane = value column j, columns 128 + 32 wh.. = tokens
+        tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
+        uint8_t *ub = sm + f.us + (uint32_t)(row >> 6) * 8192;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
+            *reinterpret_cast<uint4 *>(ub + tc::sw128(row & 63, (4 * wh + c16) * 16)) =
+                make_uint4(u[0], u[1], u[2], u[3]);
+        }
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    tc::tc_fence_after_sync();
+    if (tid == 0) {
+        tc::bulk_s2g(rec + Record::kU, sm + f.us, 16384);
+        tc::bulk_commit();
+        const uint32_t wd = tc::smem_u32(sm + f.w);
+        const uint32_t kd = tc::smem_u32(sm + f.kht);
+        const uint32_t pd = tc::smem_u32(sm + f.pp);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem, tc::smem_desc(kd + kk * 32, 16, 1024),
+                         tc::smem_desc(wd + kk * 2048, 8192, 1024), tc::idesc_bf16(128, 128, 0, 1),
+                         kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem + 128, tc::smem_desc(pd + kk * 32, 16, 1024),
+                         tc::smem_desc(wd + kk * 2048, 8192, 1024), tc::idesc_bf16(64, 128, 0, 1),
+                         kk > 0);
+        tc::mma_commit(bar_np);
+        // the staging below reuses memory that earlier bulk stores read from
+        tc::bulk_wait_read_all();
+    }
+    {
+        tc::mbar_wait(bar_np, 0, abort, p.err, code + 1, p.spin);
+        tc::tc_fence_after_sync();
+        __syncthreads();
+        const int i = lg * 32 + lane;  // N: lane = key channel i, columns i' = 64 wh..
+        uint8_t *nb = sm + (wh ? f.n1 : f.n0);
+        float w[32];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
+#pragma unroll
+            for (int c16 = 0; c16 < 4; ++c16) {
+                uint32_t u[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(-w[c16 * 8 + 2 * e], -w[c16 * 8 + 2 * e + 1]);
+                *reinterpret_cast<uint4 *>(nb + tc::sw128(i, (q2 * 4 + c16) * 16)) =
+                    make_uint4(u[0], u[1], u[2], u[3]);
+            }
+        }
+        // P W (M = 64): row t in lanes 0..15 of lane group lg, columns split by
+        // half warps: this thread has channels 64 wh + 32 (lane / 16) .. + 31
+        const int t = 16 * lg + (lane & 15), hl = lane >> 4;
+        tc::tmem_ld16x2_x32_sync(la + 128 + 64 * wh, w);
+        uint8_t *qb = sm + f.qp + (uint32_t)wh * 8192;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+            const int cb = 4 * hl + c16;  // 16-byte chunk inside the key block
+            float q8[8];
+            qt(t, wh, cb, q8);
+            uint32_t u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                u[e] = pack_bf16x2(q8[2 * e] - w[c16 * 8 + 2 * e], q8[2 * e + 1] - w[c16 * 8 + 2 * e + 1]);
+            *reinterpret_cast<uint4 *>(qb + (uint32_t)t * 128 + ((((uint32_t)cb) ^ ((uint32_t)t & 7u)) << 4)) =
+                make_uint4(u[0], u[1], u[2], u[3]);
+        }
+    }
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+        tc::fence_proxy_async_global();  // Q~ written to the Q' slot by threads, overwritten now
+        tc::bulk_s2g(rec + Record::kBk, sm + f.n0, 16384);
+        tc::bulk_s2g(rec + Record::kBk + Record::kBlk, sm + f.n1, 16384);
+        tc::bulk_s2g(rec + Record::kBk + Record::kOut, sm + f.qp, 8192);
+        tc::bulk_s2g(rec + Record::kBk + Record::kBlk + Record::kOut, sm + f.qp + 8192, 8192);
+        tc::bulk_commit();
+        tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
+        // drain (matters only after a wait gave up): the input tiles have
+        // landed and every MMA has finished before the memory is released
+        tc::mbar_drain(bar_ld, 0, p.err, code + 2, p.spin);
+        tc::mma_commit(bar_fin);
+        tc::mbar_drain(bar_fin, 0, p.err, code + 2, p.spin);
+    }
+}
+
 __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid_constant__ TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -505,6 +680,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         tc::mbar_init(bar_wu, 1);
         tc::mbar_init(bar_ld, 1);
         tc::mbar_init(bar_ld + 1, 1);  // bar_fin
+        tc::mbar_init(bar_ld + 2, 1);  // bar_np
         *abort = 0;
         tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_ld, 10 * 8192);
@@ -596,6 +772,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w; a[4] = y.x; a[5] = y.y; a[6] = y.z; a[7] = y.w;
     };
     const bool first_half = tg < 8;
+    uint32_t khp[8][2];  // K^ of this thread's 4 tokens as bf16 pairs, per channel
+    float kh_even[8];
     // Products that only feed bf16 operands are formed in packed bf16 (two per
     // instruction): the factor is rounded to bf16 once, the product once more.
     auto to2 = [](const float *a, __nv_bfloat162 *b2) {
@@ -623,10 +801,24 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         for (int j = 0; j < 8; ++j) { E[j] = __expf(ge[j]); Hh[j] = __expf(t8[j] - ge[j]); }
         const float b = sbeta[r];
         // record: Q~ (rows 64.. of A1) and K^ (MN-major image)
+        // Q~ = e^{g} q into the Q' slot of the record (read back for Q' = Q~ - P W)
         to2(E, f2);
-        *reinterpret_cast<uint4 *>(rec + Record::kA1 + kb * 16384 + (64 + r) * 128 + sw) = mul4(qe, f2);
-        to2(Hh, f2);
-        *reinterpret_cast<uint4 *>(rec + Record::kKh + kb * 8192 + r * 128 + sw) = mul4(ke, f2);
+        *reinterpret_cast<uint4 *>(rec + Record::kBk + kb * Record::kBlk + Record::kOut + r * 128 +
+                                   sw) = mul4(qe, f2);
+        {   // K^ = e^{g_C - g} k, paired over consecutive tokens for the transposed image
+            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&ke);
+            float kh[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                kh[2 * j] = Hh[2 * j] * __low2float(k2[j]);
+                kh[2 * j + 1] = Hh[2 * j + 1] * __high2float(k2[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (e & 1) khp[j][e >> 1] = pack_bf16x2(kh_even[j], kh[j]);
+                else kh_even[j] = kh[j];
+            }
+        }
         // solve right-hand sides (MN-major: token rows, channel columns)
 #pragma unroll
         for (int j = 0; j < 8; ++j) t8[j] = b * E[j];
@@ -687,6 +879,15 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
             *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (64 + r) * 128 + sw) = mul4(qe, f2);
         }
     }
+    // K^ as rows i (channels) over the tokens: this thread's 4 tokens are 8
+    // bytes of each of its 8 channel rows
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t i = (uint32_t)(c0 + j);
+        *reinterpret_cast<uint2 *>(rec + Record::kBt + i * 128 +
+                                   ((((uint32_t)tg >> 1) ^ (i & 7u)) << 4) + 8 * (tg & 1)) =
+            make_uint2(khp[j][0], khp[j][1]);
+    }
     // A chunk whose decay inside half a chunk exceeds the factorised range is
     // recomputed exactly by the fixup kernel.
     if (__syncthreads_or(clamped) && tid == 0) p.fix_list[atomicAdd(p.fix_count, 1)] = c * H + h;
@@ -737,7 +938,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
                 *reinterpret_cast<float4 *>(As + r * kLd + sh + e) = make_float4(v[0], v[1], v[2], v[3]);
             }
         } else {
-            uint8_t *prow = sm + Prep2Smem::kTt;  // P staged where [T; 0] goes later
+            uint8_t *prow = sm + Prep2Smem::kP;  // P stays: the record's and MMA-NP's operand
 #pragma unroll
             for (int c16 = 0; c16 < 4; ++c16) {
                 uint32_t w[4];
@@ -756,7 +957,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     tc::tc_fence_before_sync();
     __syncthreads();
     if (tid == 0) {
-        tc::bulk_s2g(rec + Record::kP, sm + Prep2Smem::kTt, 8192);
+        tc::bulk_s2g(rec + Record::kBt + Record::kOut, sm + Prep2Smem::kP, 8192);
         tc::bulk_commit();
     }
 
@@ -766,10 +967,14 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         uint4 *z = reinterpret_cast<uint4 *>(sm + Prep2Smem::kTt + 8192);
         for (int i = tid; i < 8192 / 16; i += kPrep2Threads) z[i] = make_uint4(0, 0, 0, 0);
     }
-    // the staged P is read before the [T; 0] image overwrites it (the
-    // inverse's barriers order this wait before that)
-    if (tid == 0) tc::bulk_wait_read_all();
     invert_unit_lower64(As, Ts, tid);
+    {   // K^ rows back from the record (written by step 1, in L2) into the A
+        // matrix's dead memory: the A operand of MMA-NP
+        const uint4 *src = reinterpret_cast<const uint4 *>(rec + Record::kBt);
+        uint4 *dst = reinterpret_cast<uint4 *>(sm + Prep2Smem::kKhT);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[tid + kPrep2Threads * i] = src[tid + kPrep2Threads * i];
+    }
     {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
         uint8_t *tt = sm + Prep2Smem::kTt;
@@ -809,54 +1014,19 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
                          tc::smem_desc(tt + kk * 32, 16, 1024), idu, kk > 0);
         tc::mma_commit(bar_wu);
     }
-    {
-        // W: lanes 0..63 (tokens), columns 0..127 (channels 64*wh..): warps 0,1,4,5.
-        // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
-        // Both as record images in the A / T scratch, dead by now: W rows of
-        // K-block kb at 8K kb, U~^T at 16K.
-        tc::mbar_wait(bar_wu, 0, abort, p.err, 12, p.spin);
-        tc::tc_fence_after_sync();
-        const int lg = warp & 3, wh = warp >> 2;
-        const int row = lg * 32 + (tid & 31);
-        const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
-        float w[32];
-        if (lg < 2) {
-            uint8_t *a1 = sm + (uint32_t)wh * 8192;
+    FinishSmem fs;
+    fs.w = Prep2Smem::kW; fs.us = Prep2Smem::kUs; fs.kht = Prep2Smem::kKhT; fs.pp = Prep2Smem::kP;
+    fs.n0 = Prep2Smem::kN0; fs.n1 = Prep2Smem::kN1; fs.qp = Prep2Smem::kQp;
+    // Q~ of row t: written by step 1 into the record's Q' slot (read back from L2)
+    auto qt = [&](int t, int kb2, int cb, float *q8) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(
+            rec + Record::kBk + kb2 * Record::kBlk + Record::kOut + t * 128 +
+            ((((uint32_t)cb) ^ ((uint32_t)t & 7u)) << 4));
+        const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
-#pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    uint32_t u[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
-                    *reinterpret_cast<uint4 *>(a1 + tc::sw128(row, (q2 * 4 + c16) * 16)) =
-                        make_uint4(u[0], u[1], u[2], u[3]);
-                }
-            }
-        }
-        tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
-        uint8_t *uu = sm + 16384 + (uint32_t)(row >> 6) * 16384;
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            *reinterpret_cast<float4 *>(uu + u_swz(row & 63, 32 * wh + 4 * m)) =
-                make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
-        tc::bulk_s2g(rec + Record::kA1, sm, 8192);
-        tc::bulk_s2g(rec + Record::kA1 + 16384, sm + 8192, 8192);
-        tc::bulk_s2g(rec + Record::kU, sm + 16384, 32768);
-        tc::bulk_commit();
-        tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
-        // drain (matters only after a wait gave up): the input tiles have
-        // landed and every MMA has finished before the memory is released
-        tc::mbar_drain(bar_ld, 0, p.err, 13, p.spin);
-        tc::mma_commit(bar_ld + 1);
-        tc::mbar_drain(bar_ld + 1, 0, p.err, 13, p.spin);
-    }
+        for (int e = 0; e < 4; ++e) { q8[2 * e] = __low2float(x2[e]); q8[2 * e + 1] = __high2float(x2[e]); }
+    };
+    finish_record(sm, fs, tmem, rec, bar_wu, bar_ld + 2, bar_ld, bar_ld + 1, abort, p, 12, qt);
     if (warp == 0) {
         __syncwarp();
         tc::tc_fence_after_sync();
@@ -888,21 +1058,15 @@ struct GdnSmem {
     static constexpr uint32_t kG = 111616;    // fp32 g [64], beta [64]
     static constexpr uint32_t kBar = 112128;  // barriers + tmem slot + flags
     static constexpr uint32_t kBytes = kBar + 64 + 1024;
+    // Later tenants (each region is dead by then):
+    static constexpr uint32_t kP = kTw + 8192;  // 8192:  P, from the A/P read-out to MMA-NP
+    static constexpr uint32_t kKhT = 49152;     // 16384: K^ rows i, after the T images
+    static constexpr uint32_t kW = 65536;       // 16384: W bf16 image, after MMA-WU
 };
 static_assert(GdnSmem::kA == GdnSmem::kV + 16384 && GdnSmem::kT == GdnSmem::kA + 64 * kLd * 4 &&
               GdnSmem::kY == GdnSmem::kT + 64 * kLd * 4 && GdnSmem::kTw >= GdnSmem::kY + 3072 &&
               GdnSmem::kTw % 1024 == 0 && GdnSmem::kTu % 1024 == 0 &&
               GdnSmem::kG == GdnSmem::kTu + 8192, "GDN prep layout");
-
-// 8 bf16 values times one fp32 factor, rounded once.
-__device__ __forceinline__ uint4 scale8(uint4 x, float f)
-{
-    const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(f * __low2float(x2[j]), f * __high2float(x2[j]));
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
 
 __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __grid_constant__ TcParams p)
 {
@@ -931,6 +1095,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         tc::mbar_init(bar_wu, 1);
         tc::mbar_init(bar_ld, 1);
         tc::mbar_init(bar_ld + 1, 1);  // bar_fin
+        tc::mbar_init(bar_ld + 2, 1);  // bar_np
         *abort = 0;
         tc::fence_mbar_init();
         tc::mbar_arrive_expect_tx(bar_ld, 6 * 8192);
@@ -985,32 +1150,10 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         }
         tc::mma_commit(bar_ap);
     }
-    // ---- 3. record pieces that need only the gates, while the MMA runs:
-    // K^ = e^{g_C - g_s} k_s and Q~ = e^{g_r} q_r (rows 64.. of [W; Q~]) as their
-    // record images in the (still unused) A/T scratch, sent by bulk copies;
-    // gamma directly. Staging: K^ [0, 16K), Q~ of K-block kb at 16K + 8K kb.
+    // ---- 3. gamma, while the MMA runs
     uint8_t *rec = p.rec + ((size_t)c * H + h) * Record::kBytes;
-    uint8_t *stage = sm + GdnSmem::kA;
     const float gC = sg[C - 1];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int gi = tid + kGdnThreads * j;
-        const int sel = gi >> 10, r = (gi >> 4) & 63, oc = gi & 15;  // sel: k, q
-        const uint32_t kb = (uint32_t)(oc >> 3), sw = (uint32_t)(((oc & 7) ^ (r & 7)) << 4);
-        const uint4 x = *reinterpret_cast<const uint4 *>(sm + GdnSmem::kQK + kb * 16384 +
-                                                        (sel * 64 + r) * 128 + sw);
-        *reinterpret_cast<uint4 *>(stage + sel * 16384 + kb * 8192 + r * 128 + sw) =
-            scale8(x, __expf(sel == 0 ? gC - sg[r] : sg[r]));
-    }
     if (tid < D) reinterpret_cast<float *>(rec + Record::kG)[tid] = __expf(gC);
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        tc::bulk_s2g(rec + Record::kKh, stage, 16384);
-        tc::bulk_s2g(rec + Record::kA1 + 8192, stage + 16384, 8192);
-        tc::bulk_s2g(rec + Record::kA1 + 16384 + 8192, stage + 16384 + 8192, 8192);
-        tc::bulk_commit();
-    }
 
     // ---- 4. A (fp32, strictly lower, beta-scaled) and P (record) from D
     float *As = reinterpret_cast<float *>(sm + GdnSmem::kA);
@@ -1023,9 +1166,6 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         const int sh = (warp >> 2) * 32;       // first column s of this thread
         float d[32];
         tc::tmem_ld32_sync(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)sh, d);
-        // A overwrites the staged K^ / Q~: their bulk copies must have read it
-        if (tid == 0) tc::bulk_wait_read_all();
-        __syncthreads();
         if (t < C) {
             const int r = t;
             const float gr = sg[r], b = sbeta[r];
@@ -1042,7 +1182,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         } else {
             const int r = t - C;
             const float gr = sg[r];
-            uint8_t *prow = sm + GdnSmem::kTu;  // P staged where T Diag(beta) goes later
+            uint8_t *prow = sm + GdnSmem::kP;  // P stays: the record's and MMA-NP's operand
 #pragma unroll
             for (int c16 = 0; c16 < 4; ++c16) {
                 uint32_t w[4];
@@ -1061,18 +1201,12 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
     tc::tc_fence_before_sync();
     __syncthreads();
     if (tid == 0) {
-        tc::bulk_s2g(rec + Record::kP, sm + GdnSmem::kTu, 8192);
+        tc::bulk_s2g(rec + Record::kBt + Record::kOut, sm + GdnSmem::kP, 8192);
         tc::bulk_commit();
     }
 
-    // ---- 5. T = (I + A)^{-1}, then the two scaled T images
-    {   // rows 64..127 of [T Diag(beta e^g); 0] are zero
-        uint4 *z = reinterpret_cast<uint4 *>(sm + GdnSmem::kTw + 8192);
-        for (int i = tid; i < 8192 / 16; i += kGdnThreads) z[i] = make_uint4(0, 0, 0, 0);
-    }
-    // the staged P is read before the T images overwrite it (the inverse's
-    // barriers order this wait before them)
-    if (tid == 0) tc::bulk_wait_read_all();
+    // ---- 5. T = (I + A)^{-1}, then the two scaled T images (rows 64..127 of
+    // the W operand's A hold P: they only feed accumulator rows nobody reads)
     invert_unit_lower64_by_distance(As, Ts, Ys, tid);
     {
         const int r = tid >> 2, s0 = (tid & 3) * 16;
@@ -1116,54 +1250,48 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
                          tc::smem_desc(tu + kk * 32, 16, 1024), idu, kk > 0);
         tc::mma_commit(bar_wu);
     }
-    {
-        // W: lanes 0..63 (tokens), columns 0..127 (channels 64*wh..): warps 0,1,4,5.
-        // U~^T: lanes 0..127 (value columns), columns 128..191 (tokens 32*wh..): all warps.
-        // Both as record images in the [K; Q] and V buffers, dead once the MMAs
-        // are done: W rows of K-block kb at 8K kb, U~^T at 16K.
-        tc::mbar_wait(bar_wu, 0, abort, p.err, 22, p.spin);
-        tc::tc_fence_after_sync();
-        const int lg = warp & 3, wh = warp >> 2;
-        const int row = lg * 32 + lane;
-        const uint32_t la = tmem + ((uint32_t)(lg * 32) << 16);
-        float w[32];
-        if (lg < 2) {
-            uint8_t *a1 = sm + (uint32_t)wh * 8192;
+    // K^ = e^{g_C - g_t} k_t as rows i over the tokens (the record's image and
+    // MMA-NP's A operand), from the raw k tile while the MMAs run: thread ->
+    // channel i, 8 tokens of chunk cq; a warp reads one tile row per token
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                tc::tmem_ld32_sync(la + 64 * wh + 32 * q2, w);
+    for (int j = 0; j < 4; ++j) {
+        const int gi = tid + kGdnThreads * j;
+        const int cq = gi >> 7, i = gi & 127;
+        const uint32_t kb = (uint32_t)(i >> 6), ib = 2u * (uint32_t)(i & 63);
+        float kh[8];
 #pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    uint32_t u[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(w[c16 * 8 + 2 * e], w[c16 * 8 + 2 * e + 1]);
-                    *reinterpret_cast<uint4 *>(a1 + tc::sw128(row, (q2 * 4 + c16) * 16)) =
-                        make_uint4(u[0], u[1], u[2], u[3]);
-                }
-            }
+        for (int e = 0; e < 8; ++e) {
+            const int t = 8 * cq + e;
+            const __nv_bfloat16 x = *reinterpret_cast<const __nv_bfloat16 *>(
+                sm + GdnSmem::kQK + kb * 16384 + tc::sw128((uint32_t)t, ib));
+            kh[e] = __expf(gC - sg[t]) * __bfloat162float(x);
         }
-        tc::tmem_ld32_sync(la + 128 + 32 * wh, w);
-        uint8_t *uu = sm + 16384 + (uint32_t)(row >> 6) * 16384;
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-            *reinterpret_cast<float4 *>(uu + u_swz(row & 63, 32 * wh + 4 * m)) =
-                make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+        *reinterpret_cast<uint4 *>(sm + GdnSmem::kKhT + tc::sw128((uint32_t)i, 16u * (uint32_t)cq)) =
+            make_uint4(pack_bf16x2(kh[0], kh[1]), pack_bf16x2(kh[2], kh[3]),
+                       pack_bf16x2(kh[4], kh[5]), pack_bf16x2(kh[6], kh[7]));
     }
     tc::fence_proxy_async_smem();
-    tc::tc_fence_before_sync();
     __syncthreads();
     if (tid == 0) {
-        tc::bulk_s2g(rec + Record::kA1, sm, 8192);
-        tc::bulk_s2g(rec + Record::kA1 + 16384, sm + 8192, 8192);
-        tc::bulk_s2g(rec + Record::kU, sm + 16384, 32768);
+        tc::bulk_s2g(rec + Record::kBt, sm + GdnSmem::kKhT, 16384);
         tc::bulk_commit();
-        tc::bulk_wait_read_all();  // the CTA's shared memory must outlive the reads
-        // drain (matters only after a wait gave up): the input tiles have
-        // landed and every MMA has finished before the memory is released
-        tc::mbar_drain(bar_ld, 0, p.err, 23, p.spin);
-        tc::mma_commit(bar_ld + 1);
-        tc::mbar_drain(bar_ld + 1, 0, p.err, 23, p.spin);
     }
+    FinishSmem fs;
+    fs.w = GdnSmem::kW; fs.us = GdnSmem::kV; fs.kht = GdnSmem::kKhT; fs.pp = GdnSmem::kP;
+    fs.n0 = GdnSmem::kKhT; fs.n1 = GdnSmem::kW; fs.qp = GdnSmem::kTw;
+    // Q~ of row t: e^{g_t} times the raw q tile (rows 64.. of the [K; Q] buffer)
+    auto qt = [&](int t, int kb2, int cb, float *q8) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(
+            sm + GdnSmem::kQK + kb2 * 16384 + (64 + t) * 128 + ((((uint32_t)cb) ^ ((uint32_t)t & 7u)) << 4));
+        const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
+        const float et = __expf(sg[t]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            q8[2 * e] = et * __low2float(x2[e]);
+            q8[2 * e + 1] = et * __high2float(x2[e]);
+        }
+    };
+    finish_record(sm, fs, tmem, rec, bar_wu, bar_ld + 2, bar_ld, bar_ld + 1, abort, p, 22, qt);
     if (warp == 0) {
         __syncwarp();
         tc::tc_fence_after_sync();
@@ -1173,32 +1301,32 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
 
 // ------------------------------------------------------------------- carry
 // The state slice is carried transposed, S^T (64 value columns x 128 key
-// channels), so that every product of a chunk step has the slice's 64 value
-// columns on the M side, and the 64 tokens of W and of Q~ share one N = 128:
-//     MMA1  D1       = S^T . [W; Q~]^T  (64x128, K = 128)  -> (W S)^T | (Q~ S)^T
-//     MMA2  D2       = U^T . K^         (64x128, K = 64)   -> (K^^T U)^T
-//     MMA3  D1[:,64:] += U^T . P^T      (64x64,  K = 64)   -> O^T = (Q~ S + P U)^T
-// with U^T = U~^T - (W S)^T and S^T <- S^T Diag(gamma) + D2. M = 64 products
-// issue in about two thirds of the time of M = 128 ones.
+// channels). With N = K^^T W and Q' = Q~ - P W precomputed per chunk, one
+// chunk step is a single product with the slice's 64 value columns on the M
+// side:
+//     D = U~^T . [K^ | P^T]  +  S^T . [-N^T | Q'^T]       (64 x 192)
+// whose columns 0..127 are the state increment and columns 128..191 the
+// output, since U = U~ - W S gives
+//     S_next^T = S^T Diag(gamma) + D[:, :128],   O^T = scale * D[:, 128:].
+// The U~ part does not depend on S, so it is issued as soon as the record has
+// landed ("early", 4 K-steps over the tokens); the S part (8 K-steps over the
+// keys) follows the moment the state warps have written bf16 S^T. D is
+// double-buffered in TMEM, and S^T in shared memory, so the early group of
+// chunk c+1 and the state update of chunk c overlap.
 // An M = 64 accumulator keeps row m in TMEM lane 32*(m/16) + m%16; warp w reads
 // rows 16*(w%4) .. +15 with the 16x32bx2 shape, lanes 0-15 and 16-31 splitting
 // the columns. Warps 0-7 own the state: thread (w, l) keeps S^T row
-// 16*(w%4) + l%16, key channels 64*(w/4) + 32*(l/16) .. +31, in fp32 registers.
-// Warp 8 streams the records into a two-stage ring with bulk copies. Warp 9
-// issues the MMAs right after the named barrier that completes their operand.
-// Every thread of warps 0-7 and 9 meets each of these barriers once per chunk,
-// also after a wait has given up, so their generations never mix; warp 9
-// reaches them first, so the state warps do not wait there. MMA3 runs while
-// the state warps update S; its completion and the state warps' arrivals
-// release the record stage. D1 is double-buffered in TMEM. The output of chunk
-// c is read out of TMEM at the end of chunk c, once MMA3 is done and the
-// tensor pipe is idle (a TMEM load next to a running MMA slows both), and is
-// stored while MMA1 of chunk c+1 runs.
+// 16*(w%4) + l%16, key channels 64*(w/4) + 32*(l/16) .. +31, in fp32 registers,
+// and stores output tokens 32*(w/4) + 16*(l/16) .. +15 of that value column.
+// Warp 8 streams the records into a two-stage ring with bulk copies; warp 9
+// issues the MMAs. Per chunk the state warps and the MMA warp meet once at a
+// named barrier (S^T of the chunk complete), also after a wait has given up,
+// so their generations never mix.
 constexpr int kCarryThreads = 320;
 constexpr int kCarrySync = 288;      // state warps + the MMA warp
-constexpr uint32_t kTmemCols = 512;  // D1[0]: [0,128), D1[1]: [128,256), D2: [256,384)
+constexpr uint32_t kTmemCols = 512;  // D[0]: [0,192), D[1]: [256,448)
 
-enum { kErrFull = 1, kErrEmpty, kErrD1, kErrD2, kErrO, kErrDrain };
+enum { kErrFull = 1, kErrEmpty, kErrD, kErrUnused, kErrUnused2, kErrDrain };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads)
 {
@@ -1212,25 +1340,71 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CarrySmem::kBar);
     uint64_t *full = bars + 0;     // [2] record landed
-    uint64_t *empty = bars + 2;    // [2] 8 state warps + the MMA3 commit
-    uint64_t *d1_done = bars + 4;  // MMA1 completed
-    uint64_t *d2_done = bars + 5;  // MMA2 completed
-    uint64_t *o_ready = bars + 6;  // MMA3 completed: D1[c & 1] holds O^T of chunk c
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 8);
-    uint64_t *drain = bars + 9;    // all MMAs of the CTA completed
+    uint64_t *empty = bars + 2;    // [2] 8 state warps + the MMA commit
+    uint64_t *d_done = bars + 4;   // chunk's MMAs completed (one phase per chunk)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 6);
+    uint64_t *drain = bars + 7;    // all MMAs of the CTA completed
 
-    // one CTA per (sequence, head, half), sequences longest first
+    // The CTA's job: (sequence, head, half), a range of the sequence's chunks,
+    // where its state starts and ends, and whether it writes outputs.
+    //  pass 0 (no split): one CTA per (sequence, head, half), sequences longest
+    //    first; the whole sequence from S0 to S_final, with outputs.
+    //  pass 1 of a split into P segments: per (sequence, head), segment 0 from
+    //    S0 with outputs (its end state kept), and for every later segment p the
+    //    state from a zero start and the transition (the product of the chunk
+    //    steps' linear parts, carried like a state that starts at the identity
+    //    and has no U~ term), both without outputs: 2 + 4 (P - 1) CTAs.
+    //  pass 2: every segment p >= 1 again from its true entry state (the end
+    //    state of segment p - 1, combined in between), with outputs; the last
+    //    segment writes S_final: 2 (P - 1) CTAs.
     const int H = p.H;
-    const int half = blockIdx.x % kSlices;
-    const int h = (blockIdx.x / kSlices) % H;
-    const int n = p.order[blockIdx.x / (kSlices * H)];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int half, h, n, seg = 0;
+    const float *S_in;
+    float *S_out;
+    bool outputs = true, transition = false;
+    const size_t blk = (size_t)D * D;
+    auto seg_block = [&](int kind, int sp, int sn, int sh) {
+        return p.seg + ((((size_t)kind * p.nseg + sp) * p.N + sn) * H + sh) * blk;
+    };
+    if (p.pass == 0) {
+        half = blockIdx.x % kSlices;
+        h = (blockIdx.x / kSlices) % H;
+        n = p.order[blockIdx.x / (kSlices * H)];
+        S_in = p.S0 ? p.S0 + ((size_t)n * H + h) * blk : nullptr;
+        S_out = p.S_final ? p.S_final + ((size_t)n * H + h) * blk : nullptr;
+    } else if (p.pass == 1) {
+        const int Q = 2 + 4 * (p.nseg - 1), q = blockIdx.x % Q, u = blockIdx.x / Q;
+        h = u % H;
+        n = p.order[u / H];
+        if (q < 2) {
+            half = q;
+            S_in = p.S0 ? p.S0 + ((size_t)n * H + h) * blk : nullptr;
+            S_out = seg_block(2, 0, n, h);
+        } else {
+            const int r = q - 2;
+            seg = 1 + r / 4;
+            half = r & 1;
+            transition = (r >> 1) & 1;
+            outputs = false;
+            S_in = nullptr;
+            S_out = seg_block(transition ? 1 : 0, seg, n, h);
+        }
+    } else {
+        const int Q = 2 * (p.nseg - 1), q = blockIdx.x % Q, u = blockIdx.x / Q;
+        h = u % H;
+        n = p.order[u / H];
+        seg = 1 + q / 2;
+        half = q & 1;
+        S_in = seg_block(2, seg - 1, n, h);
+        S_out = (seg == p.nseg - 1 && p.S_final) ? p.S_final + ((size_t)n * H + h) * blk : nullptr;
+    }
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&full[0], 1); tc::mbar_init(&full[1], 1);
         tc::mbar_init(&empty[0], 9); tc::mbar_init(&empty[1], 9);
-        tc::mbar_init(d1_done, 1); tc::mbar_init(d2_done, 1); tc::mbar_init(o_ready, 1);
+        tc::mbar_init(d_done, 1);
         tc::mbar_init(drain, 1);
         *abort = 0;
         tc::fence_mbar_init();
@@ -1241,26 +1415,46 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     tc::tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    const int ts = p.seq_start[n], te = p.seq_start[n + 1];
-    const int c0 = p.chunk_off[n], nc = p.chunk_off[n + 1] - c0;
+    const int te = p.seq_start[n + 1];
+    int c0 = p.chunk_off[n], nc = p.chunk_off[n + 1] - c0;
+    if (p.pass != 0) {  // this segment's chunks: [nc p / P, nc (p + 1) / P)
+        const int b0 = (int)((long long)nc * seg / p.nseg);
+        const int b1 = (int)((long long)nc * (seg + 1) / p.nseg);
+        c0 += b0;
+        nc = b1 - b0;
+    }
+    // first token of the CTA's first chunk
+    const int ts = p.seq_start[n] + (c0 - p.chunk_off[n]) * C;
+    constexpr uint32_t kStageBytes = 49152 + 24576 + 8192 + 512;
 
     if (warp == 8) {
         // ---------------- producer: one record per chunk into the two-stage ring
         if (lane == 0) {
+            // Records of the chunks kAhead ahead are prefetched into L2, so that
+            // a stage's copy, issued as soon as the stage is released (about one
+            // chunk step before the MMAs need it), reads L2 rather than DRAM.
+            constexpr int kAhead = 4;
+            auto prefetch = [&](int lc) {
+                const uint8_t *rec = p.rec + ((size_t)(c0 + lc) * H + h) * Record::kBytes;
+                tc::bulk_prefetch_l2(rec, Record::kU);  // both B ranges
+                tc::bulk_prefetch_l2(rec + Record::kU + half * 8192, 8192);
+                tc::bulk_prefetch_l2(rec + Record::kG, 512);
+            };
+            for (int lc = 2; lc < nc && lc < 2 + kAhead && !p.starve; ++lc) prefetch(lc);
             int issued = 0;
             for (int lc = 0; lc < nc && !p.starve; ++lc) {
                 const int st = lc & 1;
+                if (lc + 2 + kAhead < nc) prefetch(lc + 2 + kAhead);
                 if (lc >= 2 && !tc::mbar_wait(&empty[st], ((lc >> 1) - 1) & 1, abort, p.err,
                                               kErrEmpty, p.spin))
                     break;
                 if (*abort) break;
                 const uint8_t *rec = p.rec + ((size_t)(c0 + lc) * H + h) * Record::kBytes;
                 uint8_t *sb = sm + st * CarrySmem::kStage;
-                tc::mbar_arrive_expect_tx(&full[st], 32768 + 16384 + 8192 + 16384 + 512);
-                tc::bulk_g2s(sb + CarrySmem::kA1, rec + Record::kA1, 32768, &full[st]);
-                tc::bulk_g2s(sb + CarrySmem::kKh, rec + Record::kKh, 16384, &full[st]);
-                tc::bulk_g2s(sb + CarrySmem::kP, rec + Record::kP, 8192, &full[st]);
-                tc::bulk_g2s(sb + CarrySmem::kU, rec + Record::kU + half * 16384, 16384, &full[st]);
+                tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+                tc::bulk_g2s(sb + CarrySmem::kBk, rec + Record::kBk, 49152, &full[st]);
+                tc::bulk_g2s(sb + CarrySmem::kBt, rec + Record::kBt, 24576, &full[st]);
+                tc::bulk_g2s(sb + CarrySmem::kU, rec + Record::kU + half * 8192, 8192, &full[st]);
                 tc::bulk_g2s(sb + CarrySmem::kG, rec + Record::kG, 512, &full[st]);
                 issued = lc + 1;
             }
@@ -1271,47 +1465,41 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         }
     } else if (warp == 9) {
         // ---------------- MMA issue
-        const uint32_t id1 = tc::idesc_bf16(64, 128, 0, 0);  // S^T . [W; Q~]^T
-        const uint32_t id2 = tc::idesc_bf16(64, 128, 0, 1);  // U^T . K^ (MN-major)
-        const uint32_t id3 = tc::idesc_bf16(64, 64, 0, 0);   // U^T . P^T
-        const uint32_t a_s = tc::smem_u32(sm + CarrySmem::kSt);
-        const uint32_t a_u = tc::smem_u32(sm + CarrySmem::kUt);
+        // the transition needs only the state columns and no U~ term
+        const uint32_t id = tc::idesc_bf16(64, transition ? 128 : 192, 0, 0);
+        const uint32_t a_s0 = tc::smem_u32(sm + CarrySmem::kSt);
         bool issued = false;
         for (int lc = 0; lc < nc; ++lc) {
             const int st = lc & 1;
             const uint32_t sb = tc::smem_u32(sm + st * CarrySmem::kStage);
-            const uint32_t d1 = tmem + (uint32_t)st * 128;
-            // after an abort no MMA is issued; the barriers are still met
+            const uint32_t d = tmem + (uint32_t)st * 256;
+            // after an abort no MMA is issued; the barrier is still met
             bool go = false;
-            if (lane == 0)
+            if (lane == 0) {
                 go = tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull, p.spin) &&
                      !*abort;
-            __syncwarp();
-            named_bar(1, kCarrySync);  // S^T complete
-            if (go) {
-                issued = true;
-                tc::tc_fence_after_sync();
+                if (go && !transition) {  // early: D = U~^T . [K^ | P^T]
+                    issued = true;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(d1, tc::smem_desc(a_s + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                                 tc::smem_desc(sb + CarrySmem::kA1 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                 id1, kk > 0);
-                tc::mma_commit(d1_done);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(d, tc::smem_desc(sb + CarrySmem::kU + kk * 32, 16, 1024),
+                                     tc::smem_desc(sb + CarrySmem::kBt + kk * 32, 16, 1024), id,
+                                     kk > 0);
+                }
             }
             __syncwarp();
-            named_bar(2, kCarrySync);  // U^T complete
-            if (go && !*abort) {
+            named_bar(1, kCarrySync);  // S^T of this chunk complete
+            if (lane == 0 && go && !*abort) {
+                issued = true;
                 tc::tc_fence_after_sync();
+                const uint32_t a_s = a_s0 + (uint32_t)st * 16384;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + 256, tc::smem_desc(a_u + kk * 32, 16, 1024),
-                                 tc::smem_desc(sb + CarrySmem::kKh + kk * 2048, 8192, 1024), id2, kk > 0);
-                tc::mma_commit(d2_done);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(d1 + 64, tc::smem_desc(a_u + kk * 32, 16, 1024),
-                                 tc::smem_desc(sb + CarrySmem::kP + kk * 32, 16, 1024), id3, 1);
-                tc::mma_commit(o_ready);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(d, tc::smem_desc(a_s + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                 tc::smem_desc(sb + CarrySmem::kBk + (kk >> 2) * Record::kBlk +
+                                               (kk & 3) * 32, 16, 1024),
+                                 id, (transition && kk == 0) ? 0u : 1u);
+                tc::mma_commit(d_done);
                 tc::mma_commit(&empty[st]);
             }
             __syncwarp();
@@ -1327,16 +1515,20 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
         const int lg = warp & 3, wh = warp >> 2, hl = lane >> 4;
         const int cr = 16 * lg + (lane & 15);  // S^T row: value column inside the slice
         const int kc0 = 64 * wh + 32 * hl;     // first key channel of this thread
-        const int tk0 = 32 * wh + 16 * hl;     // first token of this thread in U^T and O^T
         const uint32_t lane_base = tmem + ((uint32_t)(lg * 32) << 16);
         float S[32];
-        const size_t sbase = ((size_t)n * H + h) * D * D + (size_t)kc0 * D + half * kSlice + cr;
+        const size_t sbase = (size_t)kc0 * D + half * kSlice + cr;  // inside a (sequence, head) block
+        if (transition) {  // the identity: S^T row (half * 64 + cr) is that unit vector
 #pragma unroll
-        for (int j = 0; j < 32; ++j) S[j] = p.S0 ? p.S0[sbase + (size_t)j * D] : 0.f;
+            for (int j = 0; j < 32; ++j) S[j] = (kc0 + j == half * kSlice + cr) ? 1.f : 0.f;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) S[j] = S_in ? S_in[sbase + (size_t)j * D] : 0.f;
+        }
         // bf16 S^T row cr, channels kc0..kc0+31: 4 of the row's 8 swizzled
-        // 16-byte chunks in K-block wh
-        auto store_st = [&]() {
-            uint8_t *base = sm + CarrySmem::kSt + wh * 8192;
+        // 16-byte chunks in K-block wh of buffer `buf`
+        auto store_st = [&](int buf) {
+            uint8_t *base = sm + CarrySmem::kSt + buf * 16384 + wh * 8192;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t w[4];
@@ -1346,19 +1538,11 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
-        // Output of chunk lc: O^T rows in D1[lc & 1], columns 64..127, read into
-        // ov by read_o. store_o sends the warp's 16 value columns x 32 tokens
-        // through a 1 KB staging tile (token rows of 32 bytes, value pairs packed
-        // with one shuffle), then to o with two 16-byte stores per lane: 2 global
-        // store instructions per warp instead of 16, which would slow the
-        // concurrent MMA1.
+        // store_o sends the warp's 16 value columns x 32 tokens of chunk lc
+        // through a 1 KB staging tile (token rows of 32 bytes, value pairs
+        // packed with one shuffle), then to o with two 16-byte stores per lane.
         uint8_t *os = sm + CarrySmem::kOs + warp * 1024;
         float ov[16];
-        auto read_o = [&](int lc) {
-            tc::mbar_wait(o_ready, lc & 1, abort, p.err, kErrO, p.spin);
-            tc::tc_fence_after_sync();
-            tc::tmem_ld16x2_x16_sync(lane_base + (uint32_t)(lc & 1) * 128 + 64 + 32 * wh, ov);
-        };
         auto store_o = [&](int lc) {
             const bool odd = lane & 1;
             const int l15 = lane & 15;
@@ -1385,70 +1569,46 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
             }
             __syncwarp();
         };
-        store_st();
-        tc::fence_proxy_async_smem();
-
+        if (nc > 0) {
+            store_st(0);
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before_sync();
+            named_bar(1, kCarrySync);  // S^T of chunk 0 complete
+        }
         for (int lc = 0; lc < nc; ++lc) {
             const int st = lc & 1;
             const uint8_t *sb = sm + st * CarrySmem::kStage;
-            // A. S^T is complete: MMA1 may go
-            tc::tc_fence_before_sync();
-            named_bar(1, kCarrySync);
-            // B. previous chunk's output, while MMA1 runs
-            if (lc > 0) store_o(lc - 1);
-            // C. U^T = U~^T - (W S)^T for tokens tk0..tk0+15
+            float g[32];
             tc::mbar_wait(&full[st], (lc >> 1) & 1, abort, p.err, kErrFull, p.spin);
-            tc::mbar_wait(d1_done, lc & 1, abort, p.err, kErrD1, p.spin);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(sb + CarrySmem::kG + (kc0 + j) * 4);
+                g[j] = x.x; g[j + 1] = x.y; g[j + 2] = x.z; g[j + 3] = x.w;
+            }
+            // this warp has read its piece of the stage (gamma); the MMA
+            // warp's commit covers the operands
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[st]);
+            tc::mbar_wait(d_done, lc & 1, abort, p.err, kErrD, p.spin);
             tc::tc_fence_after_sync();
             {
-                float U[16];
-                tc::tmem_ld16x2_x16_sync(lane_base + (uint32_t)st * 128 + 32 * wh, U);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float4 ut = *reinterpret_cast<const float4 *>(
-                        sb + CarrySmem::kU + u_swz(cr, tk0 + 4 * m));
-                    U[4 * m] = ut.x - U[4 * m]; U[4 * m + 1] = ut.y - U[4 * m + 1];
-                    U[4 * m + 2] = ut.z - U[4 * m + 2]; U[4 * m + 3] = ut.w - U[4 * m + 3];
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(U[8 * q + 2 * e], U[8 * q + 2 * e + 1]);
-                    *reinterpret_cast<uint4 *>(sm + CarrySmem::kUt + tc::sw128(cr, (tk0 / 8 + q) * 16)) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before_sync();
-            named_bar(2, kCarrySync);
-            // D. S^T = S^T Diag(gamma) + D2, and its bf16 copy for the next MMA1
-            {
-                float g[32];
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sb + CarrySmem::kG + (kc0 + j) * 4);
-                    g[j] = x.x; g[j + 1] = x.y; g[j + 2] = x.z; g[j + 3] = x.w;
-                }
-                tc::mbar_wait(d2_done, lc & 1, abort, p.err, kErrD2, p.spin);
-                tc::tc_fence_after_sync();
                 float ku[32];
-                tc::tmem_ld16x2_x32_sync(lane_base + 256 + 64 * wh, ku);
+                tc::tmem_ld16x2_x32_x16_sync(lane_base + (uint32_t)st * 256 + 64 * wh, ku,
+                                             lane_base + (uint32_t)st * 256 + 128 + 32 * wh, ov);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[j] = g[j] * S[j] + ku[j];
             }
-            store_st();
-            tc::fence_proxy_async_smem();
-            // this warp has read its last piece of the stage (U~^T, gamma)
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[st]);
-            // E. this chunk's output, once MMA3 is done
-            read_o(lc);
+            if (lc + 1 < nc) {
+                store_st((lc + 1) & 1);
+                tc::fence_proxy_async_smem();
+                tc::tc_fence_before_sync();
+                named_bar(1, kCarrySync);  // S^T of chunk lc+1 complete
+            }
+            if (outputs) store_o(lc);
         }
-        if (nc > 0) store_o(nc - 1);
-        if (p.S_final) {
+        if (S_out) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) p.S_final[sbase + (size_t)j * D] = S[j];
+            for (int j = 0; j < 32; ++j) S_out[sbase + (size_t)j * D] = S[j];
         }
     }
     tc::tc_fence_before_sync();
@@ -1459,7 +1619,53 @@ __global__ void __launch_bounds__(kCarryThreads, 1) tc_carry_kernel(TcParams p)
     }
 }
 
-constexpr size_t kPrepSmem = sizeof(float) * (3 * C * (D + 1) + C * D + C * (C + 1) + C);
+// ------------------------------------------------------------------- combine
+// Between the two passes of a time split: the true end state of every segment
+// but the last, S_end(p) = Phi_p S_end(p - 1) + S0_p for p = 1 .. P - 2, in
+// fp32 (Phi_p: segment p's transition, S0_p: its state from a zero start).
+// One CTA per (sequence, head, 16 value columns); sequential over p.
+constexpr int kCombThreads = 256;
+constexpr int kCombCols = 16;
+
+__global__ void __launch_bounds__(kCombThreads) tc_combine_kernel(TcParams p)
+{
+    __shared__ float sS[D][kCombCols];
+    const int H = p.H, tiles = D / kCombCols;
+    const int tile = blockIdx.x % tiles, u = blockIdx.x / tiles;
+    const int h = u % H, n = u / H;
+    const int tid = threadIdx.x, i = tid >> 1, c8 = (tid & 1) * 8, col = tile * kCombCols + c8;
+    auto block = [&](int kind, int sp) {
+        return p.seg + ((((size_t)kind * p.nseg + sp) * p.N + n) * H + h) * (size_t)D * D;
+    };
+    {
+        const float *s0 = block(2, 0) + (size_t)i * D + col;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sS[i][c8 + e] = s0[e];
+    }
+    __syncthreads();
+    for (int sp = 1; sp + 1 < p.nseg; ++sp) {
+        const float *phi = block(1, sp) + (size_t)i * D;
+        const float *z = block(0, sp) + (size_t)i * D + col;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = z[e];
+        for (int m = 0; m < D; m += 4) {
+            const float4 f = *reinterpret_cast<const float4 *>(phi + m);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                acc[e] += f.x * sS[m][c8 + e] + f.y * sS[m + 1][c8 + e] + f.z * sS[m + 2][c8 + e] +
+                          f.w * sS[m + 3][c8 + e];
+        }
+        __syncthreads();
+        float *out = block(2, sp) + (size_t)i * D + col;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { sS[i][c8 + e] = acc[e]; out[e] = acc[e]; }
+        __syncthreads();
+    }
+}
+
+constexpr size_t kPrepSmem = sizeof(float) * (4 * C * DP + C * D + 2 * C * (C + 1) + C);
+static_assert(kPrepSmem <= 227 * 1024, "fixup shared memory");
 constexpr int kFixupBlocks = 148;
 
 }  // namespace
@@ -1504,6 +1710,21 @@ bool tc_supported(const Problem &p)
     return p.dtype == KDA_DTYPE_BF16 && p.dk == 128 && p.dv == 128;
 }
 
+int tc_auto_segments(const Problem &p)
+{
+    // Split the sequential phase in time only when few (sequence, head) chains
+    // leave most SMs idle: the first pass needs 2 + 4 (P - 1) one-SM CTAs per
+    // chain and the two passes together take about 2/P of the unsplit time, so
+    // P >= 3 within one wave of 148 SMs, and segments of at least 16 chunks.
+    const long long chains = (long long)p.N * p.H;
+    if (chains <= 0 || p.max_chunks <= 0) return 1;
+    const long long per_seq = (long long)p.max_chunks / p.N;
+    long long P = (148 / chains - 2) / 4 + 1;
+    P = P < per_seq / 16 ? P : per_seq / 16;
+    if (P > kMaxSegments) P = kMaxSegments;
+    return P >= 3 ? (int)P : 1;
+}
+
 WorkspaceLayout tc_workspace_layout(const Problem &p)
 {
     WorkspaceLayout l;
@@ -1511,6 +1732,8 @@ WorkspaceLayout tc_workspace_layout(const Problem &p)
     l.plan_bytes = align_up(kWsHeader + sizeof(int32_t) * (plan_ints(p.N) +
                                                            (size_t)p.max_chunks * p.H), 1024);
     l.chunk_bytes = (size_t)Record::kBytes * (size_t)p.H * (size_t)p.max_chunks;
+    if (p.nseg > 1)  // the time split's segment states
+        l.chunk_bytes += 3 * (size_t)p.nseg * p.N * p.H * D * D * sizeof(float);
     l.total = l.plan_bytes + l.chunk_bytes;
     return l;
 }
@@ -1537,6 +1760,9 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
     const DebugKnobs dbg = debug_knobs();
     p.spin = dbg.wait_limit ? dbg.wait_limit : tc::kSpinLimit;
     p.starve = dbg.starve_carry;
+    p.nseg = pb.nseg > 1 ? pb.nseg : 1;
+    p.pass = 0;
+    p.seg = reinterpret_cast<float *>(p.rec + (size_t)Record::kBytes * pb.H * pb.max_chunks);
 
     cudaError_t e = cudaSuccess;
     if (phases & kPhasePrepare) {
@@ -1580,9 +1806,29 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
         e = cudaFuncSetAttribute(tc_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)CarrySmem::kBytes);
         if (e != cudaSuccess) return e;
-        tc_carry_kernel<<<(unsigned)(pb.N * pb.H * kSlices), kCarryThreads, CarrySmem::kBytes, st>>>(p);
-        note_launch();
-        e = cudaGetLastError();
+        const unsigned chains = (unsigned)(pb.N * pb.H);
+        if (p.nseg == 1) {
+            tc_carry_kernel<<<chains * kSlices, kCarryThreads, CarrySmem::kBytes, st>>>(p);
+            note_launch();
+            e = cudaGetLastError();
+        } else {
+            p.pass = 1;
+            tc_carry_kernel<<<chains * (2 + 4 * (p.nseg - 1)), kCarryThreads, CarrySmem::kBytes,
+                              st>>>(p);
+            note_launch();
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            if (p.nseg > 2) {
+                tc_combine_kernel<<<chains * (D / kCombCols), kCombThreads, 0, st>>>(p);
+                note_launch();
+                e = cudaGetLastError();
+                if (e != cudaSuccess) return e;
+            }
+            p.pass = 2;
+            tc_carry_kernel<<<chains * 2 * (p.nseg - 1), kCarryThreads, CarrySmem::kBytes, st>>>(p);
+            note_launch();
+            e = cudaGetLastError();
+        }
     }
     return e;
 }

@@ -100,6 +100,14 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
                  : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (no shared-memory destination).
+// Address 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src_gmem, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src_gmem), "r"(bytes)
+                 : "memory");
+}
+
 // 3-D tiled tensor copy (TMA) global -> this CTA's shared memory, completing
 // its bytes on an mbarrier; no multicast. `tmap` is the generic address of a
 // CUtensorMap in kernel-parameter space (a __grid_constant__ argument);
@@ -154,6 +162,13 @@ __device__ __forceinline__ void cp_async_wait_all()
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's generic-proxy global-memory accesses before its later
+// async-proxy accesses (bulk copies) of the same addresses.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- TMEM
@@ -228,6 +243,27 @@ __device__ __forceinline__ void tmem_ld16x2_x32_sync(uint32_t taddr, float *v)
                  : "r"(taddr) : "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Two loads of an M = 64 accumulator's rows with the 16x32bx2 shape (32 and 16
+// columns per half warp), then one wait: thread l < 16 receives columns
+// [col, col+N) of lane (lane base) + l, thread l >= 16 the columns [col+N, col+2N)
+// of lane (lane base) + l - 16, for (a, N = 32) into va and (b, N = 16) into vb.
+__device__ __forceinline__ void tmem_ld16x2_x32_x16_sync(uint32_t a, float *va, uint32_t b, float *vb)
+{
+    uint32_t r[48];
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32"
+                 " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%48], 32;\n\t"
+                 "tcgen05.ld.sync.aligned.16x32bx2.x16.b32"
+                 " {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47}, [%49], 16;\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+                   "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47])
+                 : "r"(a), "r"(b) : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) va[i] = __uint_as_float(r[i]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) vb[i] = __uint_as_float(r[32 + i]);
 }
 
 // ---------------------------------------------------------------- MMA

@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
 
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
-ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2}
+ALGOS = {"auto": 0, "simt": 1, "tcgen05": 2, "tcgen05_sequential": 3}
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
           3: "KDA_ERR_ALIGNMENT", 4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA",
           6: "KDA_ERR_DEVICE_STATUS"}
@@ -61,12 +61,14 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_fwd_workspace_size.argtypes = [_i] * 7
         L.kda_chunk_fwd_workspace_size_ex.restype = _sz
         L.kda_chunk_fwd_workspace_size_ex.argtypes = [_i] * 8
+        L.kda_chunk_fwd_timesplit_workspace_size.restype = _sz
+        L.kda_chunk_fwd_timesplit_workspace_size.argtypes = [_i] * 8
         common = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
                   _vp, _vp, _vp, _sz]
         L.kda_chunk_fwd.restype = _i
         L.kda_chunk_fwd.argtypes = common + [_vp]
         for fn in ("kda_chunk_fwd_ex", "kda_chunk_fwd_prepare", "kda_chunk_fwd_carry",
-                   "kda_gdn_chunk_fwd", "kda_gdn_chunk_fwd_prepare"):
+                   "kda_gdn_chunk_fwd", "kda_gdn_chunk_fwd_prepare", "kda_chunk_fwd_timesplit"):
             getattr(L, fn).restype = _i
             getattr(L, fn).argtypes = common + [_i, _vp]
         L.kda_decode_step.restype = _i
@@ -228,6 +230,29 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None
     """
     return ChunkFwdCall(q, k, v, log_alpha, beta, S0, cu_seqlens, scale, output_final_state,
                         workspace, o, S_final, algo).run(stream)
+
+
+def kda_chunk_fwd_timesplit(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=None,
+                            segments=0, output_final_state=True, workspace=None, o=None,
+                            S_final=None, stream=None):
+    """Tensor-core prefill with the sequential phase split into ``segments``
+    time segments per sequence (C: ``kda_chunk_fwd_timesplit``; 0 = automatic,
+    1 = no split). bf16, dk = dv = 128. Arguments and results as
+    :func:`kda_chunk_fwd`."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    n_seqs = cu_seqlens.shape[0] - 1 if cu_seqlens is not None else 0
+    need = int(lib().kda_chunk_fwd_timesplit_workspace_size(B, T, H, dk, dv, n_seqs, _dt(q),
+                                                            int(segments)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    call = ChunkFwdCall(q, k, v, log_alpha, beta, S0, cu_seqlens, scale, output_final_state,
+                        workspace, o, S_final, "tcgen05")
+    args = call.args[:-1]  # the algo is replaced by the segment count
+    st = lib().kda_chunk_fwd_timesplit(*args, int(segments), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_chunk_fwd_timesplit", st)
+    return call.o, call.S_final
 
 
 def kda_chunk_fwd_prepare(*args, stream=None, **kwargs) -> ChunkFwdCall:

@@ -71,7 +71,8 @@ typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype_t;
 typedef enum {
     KDA_ALGO_AUTO = 0,    /* tcgen05 path when supported, else SIMT */
     KDA_ALGO_SIMT = 1,    /* fp32 CUDA-core path: any supported dtype and size */
-    KDA_ALGO_TCGEN05 = 2  /* tensor-core path: bf16, dk = dv = 128 only */
+    KDA_ALGO_TCGEN05 = 2, /* tensor-core path: bf16, dk = dv = 128 only */
+    KDA_ALGO_TCGEN05_SEQUENTIAL = 3  /* tensor-core path without the time split */
 } kda_algo_t;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -152,13 +153,48 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtyp
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /* kda_chunk_fwd with an explicit algorithm choice (kda_algo_t). Asking for
- * KDA_ALGO_TCGEN05 on a problem it does not support returns KDA_ERR_UNSUPPORTED. */
+ * KDA_ALGO_TCGEN05 on a problem it does not support returns KDA_ERR_UNSUPPORTED.
+ * On the tensor-core path (AUTO and TCGEN05) the sequential phase is split in
+ * time when a problem has so few (sequence, head) chains that most SMs would
+ * idle (see kda_chunk_fwd_timesplit); KDA_ALGO_TCGEN05_SEQUENTIAL never splits. */
 kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
                               const float *log_alpha, const float *beta, const float *S0,
                               const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
                               int dk, int dv, float scale, void *o, float *S_final,
                               void *workspace, size_t workspace_bytes, int algo,
                               void *stream);
+
+/*
+ * Chunked prefill on the tensor-core path (bf16, dk = dv = 128) with the
+ * sequential phase split into `segments` time segments per sequence, so that
+ * a long sequence with few heads keeps more SMs busy. The
+ * sequential chunk walk of one (sequence, head) only runs on as many SMs as
+ * there are 64-column halves of its state; the split runs it in two parallel
+ * passes instead. Pass 1: segment 0 from S0 with outputs, and for every later
+ * segment the state from a zero start and the segment's transition (the
+ * product of the chunk steps' linear parts, a 128 x 128 matrix carried like a
+ * state that starts at the identity). A combine kernel then forms each
+ * segment's true entry state in fp32 (end = transition x entry + zero-start
+ * state). Pass 2: every later segment again from its entry state, with
+ * outputs. Results equal kda_chunk_fwd_ex's up to rounding. The recurrence is
+ * the one of the "Kimi Linear" juejin.cn page, section 三 5️⃣; the pages give no
+ * time split (the chunk-parallel form is section 三 2️⃣'s remark).
+ *   segments   0: choose automatically (as KDA_ALGO_TCGEN05), 1: no split,
+ *              2..64: that many segments per sequence (sequences with fewer
+ *              chunks get empty segments)
+ * Other arguments, layouts and errors as kda_chunk_fwd_ex; the workspace is
+ * kda_chunk_fwd_timesplit_workspace_size bytes (it grows by 192 KB per segment,
+ * sequence and head). Unsupported problems return KDA_ERR_UNSUPPORTED.
+ */
+size_t kda_chunk_fwd_timesplit_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                              kda_dtype_t qkv_dtype, int segments);
+kda_status_t kda_chunk_fwd_timesplit(const void *q, const void *k, const void *v,
+                                     kda_dtype_t qkv_dtype, const float *log_alpha,
+                                     const float *beta, const float *S0,
+                                     const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                                     int dk, int dv, float scale, void *o, float *S_final,
+                                     void *workspace, size_t workspace_bytes, int segments,
+                                     void *stream);
 
 /*
  * The two phases of kda_chunk_fwd_ex, exported separately (same arguments, same

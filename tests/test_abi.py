@@ -209,3 +209,30 @@ def test_launch_count_and_debug_knobs(L):
     assert L.kda_launch_count() == before
     assert L.kda_debug_set_wait_limit(1000, 1) == 0
     assert L.kda_debug_set_wait_limit(0, 0) == 0
+
+
+def _split_call(L, segments, **kw):
+    f = _fake()
+    a = dict(dt=1, dk=128, ws=f, ws_bytes=1 << 40)
+    a.update(kw)
+    return L.kda_chunk_fwd_timesplit(f, f, f, a["dt"], f, f, None, None, 0, 1, 4096, 4,
+                                     a["dk"], a["dk"], 0.1, f, None, a["ws"], a["ws_bytes"],
+                                     segments, None)
+
+
+@pytest.mark.parametrize("segments,kw,status", [
+    (-1, {}, 1), (65, {}, 1),                 # segment count outside 0..64
+    (3, dict(dt=0), 2), (3, dict(dk=64), 2),  # not a tensor-core problem
+    (3, dict(ws_bytes=1024), 4),              # workspace too small
+])
+def test_timesplit_rejects(L, segments, kw, status):
+    assert _split_call(L, segments, **kw) == status
+
+
+def test_timesplit_workspace_grows_with_segments(L):
+    f = L.kda_chunk_fwd_timesplit_workspace_size
+    one, four = f(1, 4096, 4, 128, 128, 0, 1, 1), f(1, 4096, 4, 128, 128, 0, 1, 4)
+    assert one > 0 and four - one == 3 * 4 * 1 * 4 * 128 * 128 * 4
+    assert f(1, 4096, 4, 128, 128, 0, 1, 65) == 0 and f(1, 4096, 4, 64, 64, 0, 1, 2) == 0
+    # the sequential algorithm never reserves segment states
+    assert L.kda_chunk_fwd_workspace_size_ex(1, 4096, 4, 128, 128, 0, 1, 3) == one
