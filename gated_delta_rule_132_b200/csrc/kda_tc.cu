@@ -245,10 +245,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams
 
 // ------------------------------------------------------------------- prep
 // Tensor-core prep. Per chunk and head (256 threads):
-//  1. Each thread owns 2 key channels x 16 tokens: loads q, k, v, log_alpha,
-//     forms the in-chunk cumulative log-decay g (quarter totals exchanged in
-//     shared memory), E_r = e^{g_r} and H_r = e^{g_C - g_r}, and writes Q~ and K^
-//     to the record and the MMA operands below to shared memory.
+//  1. Each thread owns 8 key channels x 4 tokens: loads q, k, v, log_alpha (TMA
+//     tiles), forms the in-chunk cumulative log-decay g (token-group totals
+//     exchanged in shared memory), E_r = e^{g_r} and H_r = e^{g_C - g_r}, writes
+//     K^ = H k to the record (as rows over the tokens) and Q~ = E q to the
+//     record's Q' slot, and the MMA operands below to shared memory.
 //  2. The intra-chunk matrices A and P need e^{g_r - g_s} inside a contraction
 //     over channels, so it is split into a row factor and a column factor
 //     around a reference token: rows/cols of the first half use g_15, rows of
@@ -258,13 +259,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams
 //     A (from k rows) and P (from q rows). Every factor is <= 1 except within a
 //     half, where it is bounded by the decay across at most 32 tokens; a chunk
 //     that would exceed e^80 there is listed for the exact fixup kernel.
-//  3. T = (I + A)^{-1} in fp32 by blocks of 16: the four diagonal blocks by
-//     substitution, then the off-diagonal blocks by distance,
-//     T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, as 16x16 products on all threads.
-//  4. W = [T; 0] (128x64) . beta K~ (64x128), whose accumulator rows 0..63 are
+//  3. T = (I + A)^{-1} in fp32 by blocks of 16: a 2x2 block inverse of 32-row
+//     blocks over 16-row ones (invert_unit_lower64).
+//  4. W = [T; P] (128x64) . beta K~ (64x128), whose accumulator rows 0..63 are
 //     the 64 tokens, and U~^T = (beta V)^T (128x64) . T^T (64x64), whose rows
 //     are the 128 value columns: two MMA groups on the same operand images.
-//  5. Everything goes to the record in the carry kernel's operand layouts.
+//  5. N = K^^T W and P W (finish_record): the reference-31 rows of step 2's B
+//     operand, k_s e^{g_31 - g_s} for every token s, are K^ up to the channel
+//     factor e^{g_C - g_31}, so they serve as the A operand of N and the factor
+//     scales N's rows; Q' = Q~ - P W with Q~ read back from the record.
+//  6. Everything goes to the record in the carry kernel's operand layouts.
 constexpr int kPrep2Threads = 256;
 
 constexpr uint32_t kLdBytes = 68 * 4;  // one row of the fp32 A / T matrices (kLd floats)
@@ -273,28 +277,33 @@ struct Prep2Smem {
     static constexpr uint32_t kAop = 0;        // 32768: [kb][128 rows][128B]
     static constexpr uint32_t kA = 0;          // fp32 A [64][kLd], after MMA-AP
     static constexpr uint32_t kBop = 32768;    // 24576: [kb][96 rows][128B]
-    static constexpr uint32_t kT = 32768;      // fp32 T [64][kLd], after MMA-AP
     static constexpr uint32_t kBK = 57344;     // 16384: (beta K~) MN-major image
     static constexpr uint32_t kBV = 73728;     // 16384: (beta V) MN-major image (follows BK)
-    static constexpr uint32_t kTt = 90112;     // 16384: [T; 0], K-major rows r
-    // During step 1 the [T; 0] buffer is free: it holds the token-group totals
-    // and the per-channel constants (its zero rows are written after step 2).
+    static constexpr uint32_t kTt = 90112;     // 8192:  [T; P], K-major rows r (P from 8 KB on)
+    // During step 1 the [T; P] buffer is free: it holds the token-group totals
+    // and the per-channel constants.
     static constexpr uint32_t kTot = kTt;          // 8192:  token-group totals [16][128]
     static constexpr uint32_t kCst = kTt + 8192;   // 3584:  per-channel constants [7][128]
     static constexpr uint32_t kB = 106496;     // 256:   beta [64]
     static constexpr uint32_t kBar = 106752;   // barriers + tmem slot + flags
-    static constexpr uint32_t kBytes = kBar + 64 + 1024;
+    static constexpr uint32_t kF = 106816;     // 512:   e^{g_C - g_31} per channel
+    static constexpr uint32_t kBytes = kF + 512 + 1024;
     // Later tenants of the same memory (each region is dead by then):
-    static constexpr uint32_t kKhT = 0;        // 16384: K^ as rows i over the tokens, after the inverse
-    static constexpr uint32_t kP = 18432;      // 8192:  P (K-major rows t), from the A/P read-out on
-    static constexpr uint32_t kW = 32768;      // 16384: W bf16 MN-major image, after MMA-WU
-    static constexpr uint32_t kQp = 32768;     // 16384: Q' staging (2 key blocks of 8 KB), after MMA-NP
+    static constexpr uint32_t kT = 17408;      // fp32 T [64][kLd], after MMA-AP (over the
+                                               // first key block's reference-15 rows)
+    static constexpr uint32_t kKh = 36864;     // the reference-31 rows of the B operand: k e^{g_31 - g}
+                                               // for tokens 0..63, per key block (12 KB apart);
+                                               // A of MMA-NP until it completes
+    static constexpr uint32_t kP = kTt + 8192; // 8192:  P (K-major rows t), from the A/P read-out on
+    static constexpr uint32_t kW = 0;          // 16384: W bf16 MN-major image, after MMA-WU
+    static constexpr uint32_t kQp = 0;         // 16384: Q' staging (2 key blocks of 8 KB), after MMA-NP
     static constexpr uint32_t kN0 = 57344;     // 16384: -N staging, key block 0, after MMA-WU
     static constexpr uint32_t kUs = 73728;     // 16384: U~^T bf16 staging, after MMA-WU
-    static constexpr uint32_t kN1 = 90112;     // 16384: -N staging, key block 1, after MMA-WU
+    static constexpr uint32_t kN1 = 90112;     // 16384: -N staging, key block 1, after MMA-NP
 };
-static_assert(Prep2Smem::kP >= 64 * kLdBytes && Prep2Smem::kP + 8192 <= Prep2Smem::kBop,
-              "P lives between the fp32 A matrix and the B operand");
+static_assert(Prep2Smem::kT == 64 * kLdBytes && Prep2Smem::kT + 64 * kLdBytes <= Prep2Smem::kKh &&
+              Prep2Smem::kKh == Prep2Smem::kBop + 32 * 128 && Prep2Smem::kKh % 1024 == 0,
+              "T lies between A and the reference-31 rows it must not touch");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 {
@@ -505,7 +514,11 @@ __device__ __forceinline__ void invert_unit_lower64_by_distance(const float *As,
 struct FinishSmem {
     uint32_t w;     // 16384: W bf16 MN-major image (B of MMA-NP)
     uint32_t us;    // 16384: U~^T bf16 staging
-    uint32_t kht;   // 16384: K^ rows i over the tokens (A of MMA-NP), already in place
+    uint32_t kh;    // K^ (or a per-channel multiple of it) over the tokens, already in
+                    // place: the A operand of MMA-NP
+    uint32_t kh_lbo;  // 0: K-major rows i (16 KB); else MN-major token rows, key
+                      // blocks kh_lbo bytes apart
+    uint32_t kh_scale;  // 0, or fp32 [128]: K^ row i = kh_scale[i] x the operand's row i
     uint32_t pp;    // 8192:  P rows t (A of MMA-NP), already in place
     uint32_t n0;    // 16384: -N staging, key block 0 (after MMA-NP)
     uint32_t n1;    // 16384: -N staging, key block 1 (after MMA-NP)
@@ -513,19 +526,22 @@ struct FinishSmem {
 };
 
 // The end of both prep kernels, once the W and U~^T MMAs (TMEM columns 0..127
-// lanes 0..63, and columns 128..191 lanes 0..127) are committed to bar_wu and K^
-// and P are in shared memory:
+// lanes 0..63, and columns 128..191 lanes 0..127) are committed to bar_wu and the
+// K^ operand and P are in shared memory:
 //   1. W -> bf16 MN-major image; U~^T -> bf16 rows j of its half, sent to the record;
 //   2. MMA-NP: N = K^^T W (M = 128, columns 0..127) and P W (M = 64, columns 128..255);
-//   3. -N and Q' = Q~ - P W (Q~ from qt(t, key block, chunk) as 8 floats) as record
-//      images, sent with bulk stores; then every copy and MMA is drained.
+//   3. -N and Q' = Q~ - P W as record images, sent with bulk stores; then every
+//      copy and MMA is drained.
+// Q~ of token t comes from qload(t, key block, half warp, raw[4]) (the 4
+// 16-byte chunks 4 hl .. 4 hl + 3 of the block, issued before the MMA-NP wait)
+// and qconv(t, raw chunk, q8) (8 floats).
 // Ends with the CTA's asynchronous work finished (TMEM may be released).
-template <typename QtFn>
+template <typename QLoad, typename QConv>
 __device__ __forceinline__ void finish_record(uint8_t *sm, const FinishSmem &f, uint32_t tmem,
                                               uint8_t *rec, uint64_t *bar_wu, uint64_t *bar_np,
                                               uint64_t *bar_ld, uint64_t *bar_fin,
                                               volatile int *abort, const TcParams &p, int code,
-                                              QtFn qt)
+                                              QLoad qload, QConv qconv)
 {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int lg = warp & 3, wh = warp >> 2;
@@ -570,13 +586,15 @@ __device__ __forceinline__ void finish_record(uint8_t *sm, const FinishSmem &f, 
         tc::bulk_s2g(rec + Record::kU, sm + f.us, 16384);
         tc::bulk_commit();
         const uint32_t wd = tc::smem_u32(sm + f.w);
-        const uint32_t kd = tc::smem_u32(sm + f.kht);
+        const uint32_t kd = tc::smem_u32(sm + f.kh);
         const uint32_t pd = tc::smem_u32(sm + f.pp);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem, tc::smem_desc(kd + kk * 32, 16, 1024),
-                         tc::smem_desc(wd + kk * 2048, 8192, 1024), tc::idesc_bf16(128, 128, 0, 1),
-                         kk > 0);
+            tc::mma_bf16(tmem,
+                         f.kh_lbo ? tc::smem_desc(kd + kk * 2048, f.kh_lbo, 1024)
+                                  : tc::smem_desc(kd + kk * 32, 16, 1024),
+                         tc::smem_desc(wd + kk * 2048, 8192, 1024),
+                         tc::idesc_bf16(128, 128, f.kh_lbo ? 1 : 0, 1), kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
             tc::mma_bf16(tmem + 128, tc::smem_desc(pd + kk * 32, 16, 1024),
@@ -586,11 +604,16 @@ __device__ __forceinline__ void finish_record(uint8_t *sm, const FinishSmem &f, 
         // the staging below reuses memory that earlier bulk stores read from
         tc::bulk_wait_read_all();
     }
+    // Q~ of this thread's token, fetched while MMA-NP runs
+    const int t = 16 * lg + (lane & 15), hl = lane >> 4;
+    uint4 qraw[4];
+    qload(t, wh, hl, qraw);
     {
         tc::mbar_wait(bar_np, 0, abort, p.err, code + 1, p.spin);
         tc::tc_fence_after_sync();
         __syncthreads();
         const int i = lg * 32 + lane;  // N: lane = key channel i, columns i' = 64 wh..
+        const float ns = f.kh_scale ? -reinterpret_cast<const float *>(sm + f.kh_scale)[i] : -1.f;
         uint8_t *nb = sm + (wh ? f.n1 : f.n0);
         float w[32];
 #pragma unroll
@@ -600,21 +623,21 @@ __device__ __forceinline__ void finish_record(uint8_t *sm, const FinishSmem &f, 
             for (int c16 = 0; c16 < 4; ++c16) {
                 uint32_t u[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) u[e] = pack_bf16x2(-w[c16 * 8 + 2 * e], -w[c16 * 8 + 2 * e + 1]);
+                for (int e = 0; e < 4; ++e)
+                    u[e] = pack_bf16x2(ns * w[c16 * 8 + 2 * e], ns * w[c16 * 8 + 2 * e + 1]);
                 *reinterpret_cast<uint4 *>(nb + tc::sw128(i, (q2 * 4 + c16) * 16)) =
                     make_uint4(u[0], u[1], u[2], u[3]);
             }
         }
         // P W (M = 64): row t in lanes 0..15 of lane group lg, columns split by
-        // half warps: this thread has channels 64 wh + 32 (lane / 16) .. + 31
-        const int t = 16 * lg + (lane & 15), hl = lane >> 4;
+        // half warps: this thread has channels 64 wh + 32 hl .. + 31
         tc::tmem_ld16x2_x32_sync(la + 128 + 64 * wh, w);
         uint8_t *qb = sm + f.qp + (uint32_t)wh * 8192;
 #pragma unroll
         for (int c16 = 0; c16 < 4; ++c16) {
             const int cb = 4 * hl + c16;  // 16-byte chunk inside the key block
             float q8[8];
-            qt(t, wh, cb, q8);
+            qconv(t, qraw[c16], q8);
             uint32_t u[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -750,6 +773,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         cst[4 * D + tid] = __expf(-g31);
         cst[5 * D + tid] = __expf(g15 - gC);
         cst[6 * D + tid] = __expf(g31 - gC);
+        reinterpret_cast<float *>(sm + Prep2Smem::kF)[tid] = __expf(gC - g31);
         reinterpret_cast<float *>(p.rec + ((size_t)c * H + h) * Record::kBytes + Record::kG)[tid] =
             __expf(gC);
     }
@@ -961,21 +985,10 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         tc::bulk_commit();
     }
 
-    // ---- 3. T = (I + A)^{-1} by 16x16 blocks
-    {   // rows 64..127 of the [T; 0] operand are zero (this memory held the
-        // step-1 scratch until now)
-        uint4 *z = reinterpret_cast<uint4 *>(sm + Prep2Smem::kTt + 8192);
-        for (int i = tid; i < 8192 / 16; i += kPrep2Threads) z[i] = make_uint4(0, 0, 0, 0);
-    }
+    // ---- 3. T = (I + A)^{-1} by 16x16 blocks (rows 64..127 of the W operand
+    // [T; P] hold P: they only feed accumulator rows nobody reads)
     invert_unit_lower64(As, Ts, tid);
-    {   // K^ rows back from the record (written by step 1, in L2) into the A
-        // matrix's dead memory: the A operand of MMA-NP
-        const uint4 *src = reinterpret_cast<const uint4 *>(rec + Record::kBt);
-        uint4 *dst = reinterpret_cast<uint4 *>(sm + Prep2Smem::kKhT);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[tid + kPrep2Threads * i] = src[tid + kPrep2Threads * i];
-    }
-    {   // [T; 0] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
+    {   // [T; P] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
         uint8_t *tt = sm + Prep2Smem::kTt;
 #pragma unroll
@@ -1015,18 +1028,26 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         tc::mma_commit(bar_wu);
     }
     FinishSmem fs;
-    fs.w = Prep2Smem::kW; fs.us = Prep2Smem::kUs; fs.kht = Prep2Smem::kKhT; fs.pp = Prep2Smem::kP;
+    fs.w = Prep2Smem::kW; fs.us = Prep2Smem::kUs; fs.pp = Prep2Smem::kP;
+    // K^ = e^{g_C - g_31} (k e^{g_31 - g}): the B operand's reference-31 rows times a
+    // per-channel factor, which scales the rows of N = K^^T W
+    fs.kh = Prep2Smem::kKh; fs.kh_lbo = 12288; fs.kh_scale = Prep2Smem::kF;
     fs.n0 = Prep2Smem::kN0; fs.n1 = Prep2Smem::kN1; fs.qp = Prep2Smem::kQp;
     // Q~ of row t: written by step 1 into the record's Q' slot (read back from L2)
-    auto qt = [&](int t, int kb2, int cb, float *q8) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(
-            rec + Record::kBk + kb2 * Record::kBlk + Record::kOut + t * 128 +
-            ((((uint32_t)cb) ^ ((uint32_t)t & 7u)) << 4));
+    auto qload = [&](int t, int kb2, int hl, uint4 *raw) {
+        const uint8_t *row = rec + Record::kBk + kb2 * Record::kBlk + Record::kOut + t * 128;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16)
+            raw[c16] = *reinterpret_cast<const uint4 *>(
+                row + ((((uint32_t)(4 * hl + c16)) ^ ((uint32_t)t & 7u)) << 4));
+    };
+    auto qconv = [&](int, const uint4 &x, float *q8) {
         const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
 #pragma unroll
         for (int e = 0; e < 4; ++e) { q8[2 * e] = __low2float(x2[e]); q8[2 * e + 1] = __high2float(x2[e]); }
     };
-    finish_record(sm, fs, tmem, rec, bar_wu, bar_ld + 2, bar_ld, bar_ld + 1, abort, p, 12, qt);
+    finish_record(sm, fs, tmem, rec, bar_wu, bar_ld + 2, bar_ld, bar_ld + 1, abort, p, 12, qload,
+                  qconv);
     if (warp == 0) {
         __syncwarp();
         tc::tc_fence_after_sync();
@@ -1277,12 +1298,18 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         tc::bulk_commit();
     }
     FinishSmem fs;
-    fs.w = GdnSmem::kW; fs.us = GdnSmem::kV; fs.kht = GdnSmem::kKhT; fs.pp = GdnSmem::kP;
+    fs.w = GdnSmem::kW; fs.us = GdnSmem::kV; fs.pp = GdnSmem::kP;
+    fs.kh = GdnSmem::kKhT; fs.kh_lbo = 0; fs.kh_scale = 0;
     fs.n0 = GdnSmem::kKhT; fs.n1 = GdnSmem::kW; fs.qp = GdnSmem::kTw;
     // Q~ of row t: e^{g_t} times the raw q tile (rows 64.. of the [K; Q] buffer)
-    auto qt = [&](int t, int kb2, int cb, float *q8) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(
-            sm + GdnSmem::kQK + kb2 * 16384 + (64 + t) * 128 + ((((uint32_t)cb) ^ ((uint32_t)t & 7u)) << 4));
+    auto qload = [&](int t, int kb2, int hl, uint4 *raw) {
+        const uint8_t *row = sm + GdnSmem::kQK + kb2 * 16384 + (64 + t) * 128;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16)
+            raw[c16] = *reinterpret_cast<const uint4 *>(
+                row + ((((uint32_t)(4 * hl + c16)) ^ ((uint32_t)t & 7u)) << 4));
+    };
+    auto qconv = [&](int t, const uint4 &x, float *q8) {
         const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
         const float et = __expf(sg[t]);
 #pragma unroll
@@ -1291,7 +1318,8 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
             q8[2 * e + 1] = et * __high2float(x2[e]);
         }
     };
-    finish_record(sm, fs, tmem, rec, bar_wu, bar_ld + 2, bar_ld, bar_ld + 1, abort, p, 22, qt);
+    finish_record(sm, fs, tmem, rec, bar_wu, bar_ld + 2, bar_ld, bar_ld + 1, abort, p, 22, qload,
+                  qconv);
     if (warp == 0) {
         __syncwarp();
         tc::tc_fence_after_sync();
