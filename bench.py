@@ -398,6 +398,8 @@ def bench_timesplit(steps, warmup, world, rank, dev):
         del ws
     chains = SPLIT_H
     nseg = auto or 1
+    # two CTAs (one SM each, the two 64-column halves) per (sequence, head) in the
+    # walk; the split's first pass runs 2 + 4 (P - 1) per chain, its second 2 (P - 1)
     return dict(ms_seq=out["sequential"], ms_split=out["split"], segments=nseg,
                 tokens=SPLIT_T, ctas_seq=2 * chains,
                 ctas_pass1=chains * (2 + 4 * (nseg - 1)), ctas_pass2=chains * 2 * (nseg - 1))

@@ -248,8 +248,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams
 //  1. Each thread owns 8 key channels x 4 tokens: loads q, k, v, log_alpha (TMA
 //     tiles), forms the in-chunk cumulative log-decay g (token-group totals
 //     exchanged in shared memory), E_r = e^{g_r} and H_r = e^{g_C - g_r}, writes
-//     K^ = H k to the record (as rows over the tokens) and Q~ = E q to the
-//     record's Q' slot, and the MMA operands below to shared memory.
+//     K^ = H k to the record (as rows over the tokens, swapped between lane
+//     pairs so that every store is 16 bytes) and Q~ = E q to the record's Q'
+//     slot, and the MMA operands below to shared memory.
 //  2. The intra-chunk matrices A and P need e^{g_r - g_s} inside a contraction
 //     over channels, so it is split into a row factor and a column factor
 //     around a reference token: rows/cols of the first half use g_15, rows of
@@ -261,9 +262,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_fixup_kernel(TcParams
 //     that would exceed e^80 there is listed for the exact fixup kernel.
 //  3. T = (I + A)^{-1} in fp32 by blocks of 16: a 2x2 block inverse of 32-row
 //     blocks over 16-row ones (invert_unit_lower64).
-//  4. W = [T; P] (128x64) . beta K~ (64x128), whose accumulator rows 0..63 are
-//     the 64 tokens, and U~^T = (beta V)^T (128x64) . T^T (64x64), whose rows
-//     are the 128 value columns: two MMA groups on the same operand images.
+//  4. W = [T Diag(beta); P] (128x64) . K~ (64x128), whose accumulator rows
+//     0..63 are the 64 tokens, and U~^T = V^T (128x64) . (T Diag(beta))^T
+//     (64x64), whose rows are the 128 value columns: two MMA groups on the same
+//     operand images (the v tile is used as it landed).
 //  5. N = K^^T W and P W (finish_record): the reference-31 rows of step 2's B
 //     operand, k_s e^{g_31 - g_s} for every token s, are K^ up to the channel
 //     factor e^{g_C - g_31}, so they serve as the A operand of N and the factor
@@ -277,8 +279,10 @@ struct Prep2Smem {
     static constexpr uint32_t kAop = 0;        // 32768: [kb][128 rows][128B]
     static constexpr uint32_t kA = 0;          // fp32 A [64][kLd], after MMA-AP
     static constexpr uint32_t kBop = 32768;    // 24576: [kb][96 rows][128B]
-    static constexpr uint32_t kBK = 57344;     // 16384: (beta K~) MN-major image
-    static constexpr uint32_t kBV = 73728;     // 16384: (beta V) MN-major image (follows BK)
+    static constexpr uint32_t kBK = 57344;     // 16384: K~ = e^g k MN-major image
+    static constexpr uint32_t kBV = 73728;     // 16384: the v tile as landed (MN-major), A of U~^T
+    // log_alpha lands over [kBop, kBop + 32768) (the B operand and K~'s buffer
+    // are written only after every thread holds its inputs in registers)
     static constexpr uint32_t kTt = 90112;     // 8192:  [T; P], K-major rows r (P from 8 KB on)
     // During step 1 the [T; P] buffer is free: it holds the token-group totals
     // and the per-channel constants.
@@ -693,11 +697,13 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     const uint32_t ck = (uint32_t)(oc & 7);    // chunk inside the 128-byte row
 
     // The chunk's q, k, v and log_alpha arrive as ten TMA tiles (64 tokens x
-    // 128 bytes, 128-byte swizzle) in the operand buffers, which step 1 fills
-    // only after every thread holds its inputs in registers: q, k, v as
-    // [channel block of 64][64 tokens][128 B], log_alpha as [block of 32].
+    // 128 bytes, 128-byte swizzle): q, k, v as [channel block of 64][64 tokens]
+    // [128 B], log_alpha as [block of 32]. q, k and log_alpha land in operand
+    // buffers that step 1 fills only after every thread holds its inputs in
+    // registers; v lands where it stays, as the A operand of U~^T (the solve's
+    // beta is folded into T instead).
     uint8_t *in_q = sm + Prep2Smem::kAop, *in_k = sm + Prep2Smem::kAop + 16384;
-    uint8_t *in_v = sm + Prep2Smem::kBop, *in_la = sm + Prep2Smem::kBK;
+    uint8_t *in_v = sm + Prep2Smem::kBV, *in_la = sm + Prep2Smem::kBop;
     if (tid == 0) {
         tc::mbar_init(bar_ap, 1);
         tc::mbar_init(bar_wu, 1);
@@ -721,10 +727,17 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     if (tid < C) sbeta[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * H + h] : 0.f;
 
     // ---- 1. loads and the cumulative log-decay
-    uint4 qv[4], kv[4], vv[4];
+    uint4 qv[4], kv[4];
     float g[4][8];
     __syncthreads();  // the barriers are initialised
     tc::mbar_wait(bar_ld, 0, abort, p.err, 10, p.spin);
+    // rows of the v tile past the chunk's end (the next sequence, or past the
+    // tensor) must not reach the U~ product: zero them (tail chunks only)
+    for (int i = tid; i < 2 * (C - L) * 8; i += kPrep2Threads) {
+        const int b = i / ((C - L) * 8), rem = i % ((C - L) * 8);
+        *reinterpret_cast<uint4 *>(in_v + b * 8192 + (L + (rem >> 3)) * 128 + (rem & 7) * 16) =
+            make_uint4(0, 0, 0, 0);
+    }
     {
         float run[8];
 #pragma unroll
@@ -732,18 +745,17 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = tg * 4 + e;
-            uint4 q4 = make_uint4(0, 0, 0, 0), k4 = q4, v4 = q4;
+            uint4 q4 = make_uint4(0, 0, 0, 0), k4 = q4;
             float4 la0 = make_float4(0.f, 0.f, 0.f, 0.f), la1 = la0;
             if (r < L) {  // rows past the chunk's end hold the next sequence (or zero)
                 const uint32_t qo = kb * 8192 + r * 128 + ((ck ^ (uint32_t)(r & 7)) << 4);
                 q4 = *reinterpret_cast<const uint4 *>(in_q + qo);
                 k4 = *reinterpret_cast<const uint4 *>(in_k + qo);
-                v4 = *reinterpret_cast<const uint4 *>(in_v + qo);
                 const uint32_t lb = (uint32_t)(oc >> 2) * 8192 + r * 128, j0 = (uint32_t)(oc & 3) * 2;
                 la0 = *reinterpret_cast<const float4 *>(in_la + lb + ((j0 ^ (uint32_t)(r & 7)) << 4));
                 la1 = *reinterpret_cast<const float4 *>(in_la + lb + (((j0 + 1) ^ (uint32_t)(r & 7)) << 4));
             }
-            qv[e] = q4; kv[e] = k4; vv[e] = v4;
+            qv[e] = q4; kv[e] = k4;
             run[0] += la0.x; run[1] += la0.y; run[2] += la0.z; run[3] += la0.w;
             run[4] += la1.x; run[5] += la1.y; run[6] += la1.z; run[7] += la1.w;
 #pragma unroll
@@ -812,23 +824,32 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         for (int j = 0; j < 4; ++j) r2[j] = __hmul2(x2[j], f[j]);
         return r;
     };
+    // the per-channel constants this thread needs, once for its 4 tokens:
+    // g_C, and in the fast form the factors of the reference tokens (first
+    // half: e^{-g_15}, e^{g_15 - g_C}, e^{g_31 - g_C}; second half: e^{-g_31},
+    // e^{g_31 - g_C})
+    float cC[8], cx[8], cy[8], cz[8];
+    ld8(2, cC);
+    if (fast) {
+        if (first_half) { ld8(3, cx); ld8(5, cy); ld8(6, cz); }
+        else { ld8(4, cx); ld8(6, cy); }
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int r = tg * 4 + e;
         const uint32_t sw = ((ck ^ (uint32_t)(r & 7)) << 4);  // swizzled chunk offset
         const float *ge = g[e];
-        const uint4 qe = qv[e], ke = kv[e], ve = vv[e];
-        float E[8], Hh[8], t8[8];
+        const uint4 qe = qv[e], ke = kv[e];
+        float E[8], Hh[8];
         __nv_bfloat162 f2[4];
-        ld8(2, t8);  // g_C
 #pragma unroll
-        for (int j = 0; j < 8; ++j) { E[j] = __expf(ge[j]); Hh[j] = __expf(t8[j] - ge[j]); }
-        const float b = sbeta[r];
-        // record: Q~ (rows 64.. of A1) and K^ (MN-major image)
-        // Q~ = e^{g} q into the Q' slot of the record (read back for Q' = Q~ - P W)
+        for (int j = 0; j < 8; ++j) { E[j] = __expf(ge[j]); Hh[j] = __expf(cC[j] - ge[j]); }
+        // Q~ = e^{g} q into the Q' slot of the record (read back for Q' = Q~ - P W),
+        // and K~ = e^{g} k, the B operand of W = [T Diag(beta); P] K~
         to2(E, f2);
         *reinterpret_cast<uint4 *>(rec + Record::kBk + kb * Record::kBlk + Record::kOut + r * 128 +
                                    sw) = mul4(qe, f2);
+        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBK + kb * 8192 + r * 128 + sw) = mul4(ke, f2);
         {   // K^ = e^{g_C - g} k, paired over consecutive tokens for the transposed image
             const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&ke);
             float kh[8];
@@ -843,31 +864,18 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
                 else kh_even[j] = kh[j];
             }
         }
-        // solve right-hand sides (MN-major: token rows, channel columns)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) t8[j] = b * E[j];
-        to2(t8, f2);
-        *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBK + kb * 8192 + r * 128 + sw) = mul4(ke, f2);
-        {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(b, b);
-            const __nv_bfloat162 bb[4] = {b2, b2, b2, b2};
-            *reinterpret_cast<uint4 *>(sm + Prep2Smem::kBV + kb * 8192 + r * 128 + sw) = mul4(ve, bb);
-        }
         // factors for the A/P contraction: row factor (k and q rows) and the
         // column factor(s) (k rows of the B operand)
         float ref[8];
         if (first_half) {
             float c0f[8], c1f[8];
             if (fast) {
-                ld8(3, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) E[j] *= ref[j];            // e^{g_r - g_15}
-                ld8(5, ref);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) c0f[j] = Hh[j] * ref[j];   // e^{g_15 - g_r}
-                ld8(6, ref);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) c1f[j] = Hh[j] * ref[j];   // e^{g_31 - g_r}
+                for (int j = 0; j < 8; ++j) {
+                    E[j] *= cx[j];            // e^{g_r - g_15}
+                    c0f[j] = Hh[j] * cy[j];   // e^{g_15 - g_r}
+                    c1f[j] = Hh[j] * cz[j];   // e^{g_31 - g_r}
+                }
             } else {
                 ld8(0, ref);
 #pragma unroll
@@ -885,12 +893,11 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
             *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = mul4(qe, f2);
         } else {
             if (fast) {
-                ld8(4, ref);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) E[j] *= ref[j];            // e^{g_r - g_31}
-                ld8(6, ref);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) Hh[j] *= ref[j];           // e^{g_31 - g_r}
+                for (int j = 0; j < 8; ++j) {
+                    E[j] *= cx[j];            // e^{g_r - g_31}
+                    Hh[j] *= cy[j];           // e^{g_31 - g_r}
+                }
             } else {
                 ld8(1, ref);
 #pragma unroll
@@ -903,14 +910,22 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
             *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (64 + r) * 128 + sw) = mul4(qe, f2);
         }
     }
-    // K^ as rows i (channels) over the tokens: this thread's 4 tokens are 8
-    // bytes of each of its 8 channel rows
+    // K^ as rows i (channels) over the tokens. The lane 16 apart holds the
+    // same 8 channels for the next 4 tokens: the pair swaps halves so that each
+    // lane has 4 channels x 8 tokens, one 16-byte chunk of each channel row.
+    {
+        const bool odd_tg = tg & 1;
+        const uint32_t w8 = (uint32_t)tg >> 1;  // 8-token group: chunk of the row
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t i = (uint32_t)(c0 + j);
-        *reinterpret_cast<uint2 *>(rec + Record::kBt + i * 128 +
-                                   ((((uint32_t)tg >> 1) ^ (i & 7u)) << 4) + 8 * (tg & 1)) =
-            make_uint2(khp[j][0], khp[j][1]);
+        for (int j = 0; j < 4; ++j) {  // channels j (kept by even lanes) and 4 + j (odd)
+            const uint32_t k0 = odd_tg ? khp[4 + j][0] : khp[j][0];
+            const uint32_t k1 = odd_tg ? khp[4 + j][1] : khp[j][1];
+            const uint32_t r0 = __shfl_xor_sync(0xffffffffu, odd_tg ? khp[j][0] : khp[4 + j][0], 16);
+            const uint32_t r1 = __shfl_xor_sync(0xffffffffu, odd_tg ? khp[j][1] : khp[4 + j][1], 16);
+            const uint32_t i = (uint32_t)(c0 + (odd_tg ? 4 + j : j));
+            const uint4 v = odd_tg ? make_uint4(r0, r1, k0, k1) : make_uint4(k0, k1, r0, r1);
+            *reinterpret_cast<uint4 *>(rec + Record::kBt + i * 128 + ((w8 ^ (i & 7u)) << 4)) = v;
+        }
     }
     // A chunk whose decay inside half a chunk exceeds the factorised range is
     // recomputed exactly by the fixup kernel.
@@ -988,7 +1003,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     // ---- 3. T = (I + A)^{-1} by 16x16 blocks (rows 64..127 of the W operand
     // [T; P] hold P: they only feed accumulator rows nobody reads)
     invert_unit_lower64(As, Ts, tid);
-    {   // [T; P] operand rows 0..63 (K-major, element (r, s) = T[r][s], zero above)
+    {   // [T Diag(beta); P] operand rows 0..63 (K-major, element (r, s) = T[r][s] beta_s,
+        // zero above the diagonal)
         const int r = tid >> 2, s0 = (tid & 3) * 16;
         uint8_t *tt = sm + Prep2Smem::kTt;
 #pragma unroll
@@ -999,7 +1015,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
                 const int sa = s0 + h2 * 8 + 2 * e, sb2 = sa + 1;
                 const float va = sa < r ? Ts[r * kLd + sa] : (sa == r ? 1.f : 0.f);
                 const float vb = sb2 < r ? Ts[r * kLd + sb2] : (sb2 == r ? 1.f : 0.f);
-                w[e] = pack_bf16x2(va, vb);
+                w[e] = pack_bf16x2(va * sbeta[sa], vb * sbeta[sb2]);
             }
             *reinterpret_cast<uint4 *>(tt + tc::sw128(r, (s0 + h2 * 8) * 2)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
@@ -1010,7 +1026,7 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     __syncthreads();
     tc::tc_fence_after_sync();
 
-    // ---- 4. W = [T; 0] . beta K~ and U~^T = (beta V)^T . T^T
+    // ---- 4. W = [T Diag(beta); P] . K~ and U~^T = V^T . (T Diag(beta))^T
     if (tid == 0) {
         const uint32_t bk = tc::smem_u32(sm + Prep2Smem::kBK);  // 2 MN atoms (channels)
         const uint32_t bv = tc::smem_u32(sm + Prep2Smem::kBV);
