@@ -42,7 +42,7 @@ METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM pea
 # dram__bytes_write.sum of one ncu capture of each kernel on the chunked
 # workload, 4096 records per launch); traffic grows in proportion to the
 # records a launch processes. None: no capture of the current kernel yet.
-TRAFFIC_PER_RECORD = {"prepare": None, "carry": None, "gdn_prepare": None}
+TRAFFIC_PER_RECORD = {"prepare": 163_216, "carry": 113_586, "gdn_prepare": 128_306}
 # Algorithmic work of the prefill per token and head at d = 128, chunk 64: bytes
 # the operation must move (q, k, v bf16 in, log_alpha and beta fp32 in, o bf16
 # out; the states are added per sequence) and tensor-core flops of the chunked
@@ -317,7 +317,7 @@ def bench_backward(steps, warmup, world, rank, dev, T_b=BWD_T):
                 token_heads=T_b * P.H, workload=f"long_bf16_B1_H{P.H}_T{T_b}_d{P.d}")
 
 
-def bench_decode(P, warmup, world, rank, dev):
+def bench_decode(P, warmup, world, rank, dev, steps=None):
     """The decode workload as a chain of P.steps (1000) steps: every step's
     token inputs (fresh seeded q, k, v and gates per step) are generated on the
     device before the timed region, the state is carried from step to step,
@@ -326,9 +326,10 @@ def bench_decode(P, warmup, world, rank, dev):
     from gated_delta_rule_132_b200 import kda
     devs = f"cuda:{dev}"
     S0 = I.make_decode_state(P.N, P.H, P.d, P.s_std, P.seed + 1000 * rank, device=devs)
+    n_steps = P.steps if steps is None else steps
     toks = [I.make_decode_token(P.N, P.H, P.d, P.dtype, P.gate_shift,
                                 seed=P.step_seed0 + i + 100000 * rank, device=devs)
-            for i in range(P.steps)]
+            for i in range(n_steps)]
     o = torch.empty(P.N, P.H, P.d, dtype=P.dtype, device=devs)
     S = S0.clone()
     stream = torch.cuda.current_stream()
@@ -343,7 +344,7 @@ def bench_decode(P, warmup, world, rank, dev):
         kda.kda_decode_step(**toks[i], S=S, o=o)
         ev[1].record(stream)
 
-    total_ms, per = time_region(step, P.steps, stream, marks=2)
+    total_ms, per = time_region(step, n_steps, stream, marks=2)
     barrier(world)
     per = [p[0] for p in per]
     med = max_over_ranks(statistics.median(per), world)
@@ -351,8 +352,8 @@ def bench_decode(P, warmup, world, rank, dev):
     state_b = 2 * units * P.d * P.d * 4
     io_b = units * (3 * P.d * 2 + 4 * P.d + 4 + P.d * 2)
     del toks
-    return dict(ms=max_over_ranks(total_ms / P.steps, world), kern_ms=med, min_ms=min(per),
-                steps=P.steps, bytes=state_b + io_b, state_bytes=state_b)
+    return dict(ms=max_over_ranks(total_ms / n_steps, world), kern_ms=med, min_ms=min(per),
+                steps=n_steps, bytes=state_b + io_b, state_bytes=state_b)
 
 
 # The time-split prefill: one 1M-token sequence with few heads (B=1, H=4,
@@ -547,7 +548,8 @@ def run_ours(args, world, rank, dev):
                 extra[other.name] = o
                 del o["x"], o["call"]
                 torch.cuda.empty_cache()
-        dec = None if args.no_decode else bench_decode(I.DECODE, args.warmup, world, rank, dev)
+        dec = None if args.no_decode else bench_decode(I.DECODE, args.warmup, world, rank, dev,
+                                                       args.decode_steps)
         dtok = None if args.no_decode else bench_decode_tokens(
             I.DECODE, DECODE_TOKENS_T, args.steps, args.warmup, world, rank, dev)
         gdn = None if args.no_gdn else bench_gdn(pre, args.steps, args.warmup, world)
@@ -733,6 +735,8 @@ def main():
     ap.add_argument("--workload", choices=["long", "chunked", "varlen"], default="long",
                     help="prefill workload (default: the long-context one)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="chained decode steps (default: the workload's 1000)")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward (kda_chunk_bwd) measurement")
     ap.add_argument("--bwd-tokens", type=int, default=BWD_T,

@@ -97,6 +97,7 @@ struct TcParams {
     int nseg;
     int pass;          // 0: no split, 1: first pass, 2: second pass
     float *seg;
+    int T_uniform;     // sequences of T_uniform tokens each (no cu_seqlens), else 0
     int *fix_list;     // chunk * H + head, one per listed chunk
     // q, k, v and log_alpha as 3-D tensors {channel, head, token} for TMA tile
     // loads of 128 bytes of channels x 1 head x 64 tokens in the 128-byte
@@ -113,6 +114,33 @@ __device__ __forceinline__ int find_seq(const int32_t *chunk_off, int N, int c)
         if (chunk_off[mid] <= c) lo = mid; else hi = mid - 1;
     }
     return lo;
+}
+
+// Sequence, first packed token and length of global chunk c: arithmetic for
+// uniform batches, a search of the plan for packed sequences. False past the
+// last chunk.
+struct ChunkLoc {
+    int n, t0, L;
+};
+
+__device__ __forceinline__ bool locate_chunk(const TcParams &p, int c, ChunkLoc &loc)
+{
+    if (p.T_uniform > 0) {
+        const int per = (p.T_uniform + C - 1) / C;
+        const int n = c / per;
+        if (n >= p.N) return false;
+        const int lc = c - n * per;
+        loc.n = n;
+        loc.t0 = n * p.T_uniform + lc * C;
+        loc.L = min(C, p.T_uniform - lc * C);
+        return true;
+    }
+    const int n = find_seq(p.chunk_off, p.N, c);
+    if (n < 0) return false;
+    loc.n = n;
+    loc.t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
+    loc.L = min(C, p.seq_start[n + 1] - loc.t0);
+    return true;
 }
 
 // ------------------------------------------------------------------- exact fixup
@@ -142,10 +170,9 @@ __device__ void prep_exact_chunk(const TcParams &p, int c, int h, float *smem)
     float *sb = sP + C * (C + 1);   // [C]
 
     const int H = p.H;
-    const int n = find_seq(p.chunk_off, p.N, c);
-    if (n < 0) return;
-    const int t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
-    const int L = min(C, p.seq_start[n + 1] - t0);
+    ChunkLoc loc;
+    if (!locate_chunk(p, c, loc)) return;
+    const int t0 = loc.t0, L = loc.L;
     const int tid = threadIdx.x;
 
     for (int idx = tid; idx < C * D; idx += kPrepThreads) {
@@ -684,10 +711,9 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
     float *sbeta = reinterpret_cast<float *>(sm + Prep2Smem::kB);
 
     const int c = blockIdx.x, h = blockIdx.y, H = p.H;
-    const int n = find_seq(p.chunk_off, p.N, c);
-    if (n < 0) return;  // uniform over the CTA: nothing allocated yet
-    const int t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
-    const int L = min(C, p.seq_start[n + 1] - t0);
+    ChunkLoc loc;
+    if (!locate_chunk(p, c, loc)) return;  // uniform over the CTA: nothing allocated yet
+    const int t0 = loc.t0, L = loc.L;
     const int tid = threadIdx.x, warp = tid >> 5;
     // 16-byte granules: channel octet `oc` (8 channels = one 16-byte swizzle
     // chunk of a bf16 row) x token group `tg` (4 consecutive tokens)
@@ -1119,10 +1145,9 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
     float *sbeta = sg + C;
 
     const int c = blockIdx.x, h = blockIdx.y, H = p.H;
-    const int n = find_seq(p.chunk_off, p.N, c);
-    if (n < 0) return;  // uniform over the CTA: nothing allocated yet
-    const int t0 = p.seq_start[n] + (c - p.chunk_off[n]) * C;
-    const int L = min(C, p.seq_start[n + 1] - t0);
+    ChunkLoc loc;
+    if (!locate_chunk(p, c, loc)) return;  // uniform over the CTA: nothing allocated yet
+    const int t0 = loc.t0, L = loc.L;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- 1. k, q, v straight into their operand layouts: six TMA tiles of 64
@@ -1806,6 +1831,7 @@ cudaError_t launch_tc_prefill(const Problem &pb, void *workspace, int phases, cu
     p.starve = dbg.starve_carry;
     p.nseg = pb.nseg > 1 ? pb.nseg : 1;
     p.pass = 0;
+    p.T_uniform = pb.cu_seqlens ? 0 : pb.T;
     p.seg = reinterpret_cast<float *>(p.rec + (size_t)Record::kBytes * pb.H * pb.max_chunks);
 
     cudaError_t e = cudaSuccess;
