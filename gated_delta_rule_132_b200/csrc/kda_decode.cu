@@ -8,18 +8,20 @@
 // fp32 state is read once and written once, with no second pass.
 //
 // The step is bound by HBM: 2 * dk * dv * 4 bytes of state per (sequence, head)
-// against a few hundred bytes of token data. One CTA owns one (sequence, head):
-// its 256 threads hold the whole dk x dv state in registers (float4 per thread
-// per row, a warp covering full 512-byte rows for dv = 128), issue every state
-// load before any arithmetic, reduce S'^T k and S'^T q across row groups in
-// shared memory, and stream the updated rows back. Loads and stores use the
-// evict-first cache hint: the state is touched once per call.
-//
-// Several consecutive tokens per (sequence, head) (multi-token decode, or
-// continuing a prefill by a few tokens) run in decode_tokens_kernel with the
-// state kept in registers between them: the state still crosses HBM once each
-// way, the tokens' vectors are staged in shared memory ahead of use, and each
-// token costs two CTA barriers and its own few hundred bytes.
+// against a few hundred bytes of token data. One CTA owns one (sequence, head)
+// and keeps the whole dk x dv state in registers, so the state crosses HBM once
+// each way per call, however many tokens the call carries. Loads and stores of
+// the state use the evict-first cache hint: it is touched once per call.
+//  * decode_kernel (one token): float4 per thread per row, a warp covering full
+//    512-byte rows for dv = 128; every state load is issued before any
+//    arithmetic, and S'^T k and S'^T q are summed across row groups in shared
+//    memory.
+//  * decode_tokens_kernel (T >= 2): warp w owns dv / 8 value columns over all dk
+//    key rows, lane l 4 consecutive columns (group l mod n_c of the warp's n_c
+//    groups of 4) of the rows l / n_c + m (32 / n_c). The sums over the key rows
+//    are then sums over the lanes of one column group, by recursive halving with
+//    shuffles, so a warp needs no other warp inside a token and the CTA meets at
+//    a barrier three times per block of staged tokens.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -127,19 +129,24 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     }
 }
 
-// Several tokens per call (T >= 2). The state stays in registers as in
-// decode_kernel; the tokens' vectors are staged in shared memory in blocks of
-// kTokBlock tokens with cp.async, two blocks in flight, so a token never waits
-// for a global load. When a block lands, its log-decays become decays
-// (alpha = exp(log_alpha)) and each warp forms one token's k^T q. Per token:
-// partial S'^T k and S'^T q -> barrier -> u and o per value column -> barrier
-// -> S += k u^T. The reduction and u buffers alternate between tokens, so those
-// two barriers are the only ones a token needs.
+// Several tokens per call (T >= 2). Token vectors are staged in shared memory
+// in blocks of kTokBlock tokens with cp.async, two blocks in flight, so a token
+// never waits for a global load. When a block has landed, its rows become
+// packed {alpha, k, q} per key row (alpha = exp(log_alpha)) and k^T q per token
+// (barrier); then every warp runs the block's tokens on its own columns; o goes
+// to a staging tile and leaves as full row pieces after a last barrier, when the
+// buffer is also free for block b + 2. The value columns of a head never mix,
+// so a head's 8 column slices of dv / 8 are spread over kTokParts CTAs of
+// 8 / kTokParts warps each (smaller CTAs overlap one another's loads and
+// arithmetic better).
 constexpr int kTokBlock = 8;
+constexpr int kTokParts = 1;                      // CTAs per (sequence, head)
+constexpr int kTokWarps = 8 / kTokParts;          // warps per CTA
+constexpr int kTokThreads = 32 * kTokWarps;
 
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): each lane is one ordinary fp32
-// multiply or fused multiply-add with round-to-nearest, so results equal the
-// scalar operations bit for bit, at half the instruction count.
+// multiply or fused multiply-add with round-to-nearest, at half the
+// instruction count.
 __device__ __forceinline__ uint64_t f2(float a, float b)
 {
     uint64_t r;
@@ -165,47 +172,45 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
 
 template <int DK, int DV, typename TIn>
 struct TokSmem {
-    static constexpr int CG = DV / 4, RG = kDecodeThreads / CG;
-    // one block of staged tokens
-    static constexpr size_t kLa = 0;                                         // fp32 [TB][DK] (alpha after landing)
+    // one block of staged tokens, as landed (two buffers)
+    static constexpr size_t kLa = 0;                                         // fp32 [TB][DK]
     static constexpr size_t kK = kLa + sizeof(float) * kTokBlock * DK;        // TIn [TB][DK]
     static constexpr size_t kQ = kK + sizeof(TIn) * kTokBlock * DK;          // TIn [TB][DK]
     static constexpr size_t kV = kQ + sizeof(TIn) * kTokBlock * DK;          // TIn [TB][DV]
     static constexpr size_t kB = kV + sizeof(TIn) * kTokBlock * DV;          // fp32 [TB] beta
-    static constexpr size_t kKq = kB + sizeof(float) * kTokBlock;            // fp32 [TB] k^T q
-    static constexpr size_t kBlock = (kKq + sizeof(float) * kTokBlock + 15) / 16 * 16;
-    static constexpr size_t kRed = 2 * kBlock;                               // fp32 [2][2][RG][DV]
-    static constexpr size_t kU = kRed + sizeof(float) * 2 * 2 * RG * DV;     // fp32 [2][DV]
-    static constexpr size_t kBytes = kU + sizeof(float) * 2 * DV;
+    static constexpr size_t kBlock = (kB + sizeof(float) * kTokBlock + 15) / 16 * 16;
+    // the block being computed
+    static constexpr size_t kRow = 2 * kBlock;                               // float4 [TB][DK] {alpha, k, q, 0}
+    static constexpr size_t kKq = kRow + 16 * kTokBlock * DK;                // fp32 [TB] k^T q
+    static constexpr size_t kO = kKq + sizeof(float) * kTokBlock;            // TIn [TB][DV] output rows
+    static constexpr size_t kBytes = kO + sizeof(TIn) * kTokBlock * DV;
 };
 
 template <int DK, int DV, typename TIn>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+__global__ void __launch_bounds__(kTokThreads, 2 * kTokParts)
 decode_tokens_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                      const TIn *__restrict__ v, const float *__restrict__ log_alpha,
                      const float *__restrict__ beta, float *__restrict__ S, int T, int H,
                      int gate_per_channel, float scale, TIn *__restrict__ o)
 {
     using L = TokSmem<DK, DV, TIn>;
-    constexpr int CG = L::CG, RG = L::RG, RPT = DK / RG;
-    static_assert(DK % RG == 0 && RPT >= 1, "unsupported head size");
-    static_assert(DV <= kDecodeThreads, "one value column per thread");
+    constexpr int CPW = DV / 8;                 // value columns per warp
+    constexpr int CPC = CPW * kTokWarps;        // value columns per CTA
+    constexpr int NC = CPW / 4;                 // column groups of 4 per warp
+    constexpr int LNC = NC == 4 ? 2 : NC == 2 ? 1 : 0;
+    constexpr int NR = 32 / NC;                 // row sets (lanes per column group)
+    constexpr int RPT = DK / NR;                // key rows per thread
+    static_assert(NC == 1 || NC == 2 || NC == 4, "dv / 8 must be 4, 8 or 16 columns");
+    static_assert(DK % NR == 0 && RPT >= 1, "unsupported head size");
     extern __shared__ __align__(16) uint8_t smem[];
 
-    const int unit = blockIdx.x;  // n * H + h
+    const int unit = blockIdx.x / kTokParts;  // n * H + h
+    const int part = blockIdx.x % kTokParts;  // value columns CPC part ..
     const int n = unit / H, h = unit - n * H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int cg = tid % CG, rg = tid / CG;
+    const int cc = lane & (NC - 1), rs = lane >> LNC;
+    const int c0 = CPC * part + CPW * warp + 4 * cc;  // this thread's first value column
     float *Su = S + (size_t)unit * DK * DV;
-
-    // the state as packed pairs: st[r][0] = columns (4 cg, 4 cg + 1), st[r][1] = (+2, +3)
-    uint64_t st[RPT][2];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const float4 x = __ldcs(reinterpret_cast<const float4 *>(Su + (size_t)(r * RG + rg) * DV) + cg);
-        st[r][0] = f2(x.x, x.y);
-        st[r][1] = f2(x.z, x.w);
-    }
 
     const int nblocks = (T + kTokBlock - 1) / kTokBlock;
     auto tok_index = [&](int t) { return ((size_t)n * T + t) * H + h; };  // (n, t, h)
@@ -215,7 +220,7 @@ decode_tokens_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         const int t0 = b * kTokBlock, nt = min(kTokBlock, T - t0);
         constexpr int kLaG = DK * 4 / 16, kKG = DK * (int)sizeof(TIn) / 16, kVG = DV * (int)sizeof(TIn) / 16;
         constexpr int kPer = kLaG + 2 * kKG + kVG;  // 16-byte granules per token
-        for (int g = tid; g < nt * kPer; g += kDecodeThreads) {
+        for (int g = tid; g < nt * kPer; g += kTokThreads) {
             const int tt = g / kPer, r = g % kPer;
             const size_t tok = tok_index(t0 + tt);
             const void *src;
@@ -252,94 +257,121 @@ decode_tokens_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    stage(0);
+    if (nblocks > 0) stage(0);
     if (nblocks > 1) stage(1);
 
-    float *red = reinterpret_cast<float *>(smem + L::kRed);  // [2][2][RG][DV]
-    float *su = reinterpret_cast<float *>(smem + L::kU);     // [2][DV]
+    // the state, as packed pairs: st[m][0] = columns (c0, c0 + 1), st[m][1] = (+2, +3) of
+    // key row rs + NR m
+    uint64_t st[RPT][2];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const float4 x = __ldcs(reinterpret_cast<const float4 *>(Su + (size_t)(rs + NR * m) * DV + c0));
+        st[m][0] = f2(x.x, x.y);
+        st[m][1] = f2(x.z, x.w);
+    }
+
+    float4 *rows = reinterpret_cast<float4 *>(smem + L::kRow);
+    float *skq = reinterpret_cast<float *>(smem + L::kKq);
+    TIn *so = reinterpret_cast<TIn *>(smem + L::kO);
+    // after the reduction: this lane's sum is S'^T k (bit 4 clear) or S'^T q (set)
+    // of column c0 + e; duplicates (dv < 128) write no output
+    const bool is_q = lane & 16;
+    const int e_own = ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+    const bool primary = ((lane >> LNC) & ((4 >> LNC) - 1)) == 0;
     for (int b = 0; b < nblocks; ++b) {
-        uint8_t *buf = smem + (size_t)(b & 1) * L::kBlock;
+        const uint8_t *buf = smem + (size_t)(b & 1) * L::kBlock;
         const int t0 = b * kTokBlock, nt = min(kTokBlock, T - t0);
         // this block's copies (the later block's may stay in flight)
         if (b + 1 < nblocks) asm volatile("cp.async.wait_group 1;" ::: "memory");
         else asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
-        float *sa = reinterpret_cast<float *>(buf + L::kLa);
+        const float *sa = reinterpret_cast<const float *>(buf + L::kLa);
         const TIn *sk = reinterpret_cast<const TIn *>(buf + L::kK);
         const TIn *sq = reinterpret_cast<const TIn *>(buf + L::kQ);
         const TIn *sv = reinterpret_cast<const TIn *>(buf + L::kV);
         const float *sb = reinterpret_cast<const float *>(buf + L::kB);
-        float *skq = reinterpret_cast<float *>(buf + L::kKq);
-        // decays and k^T q of the block's tokens
-        if (gate_per_channel) {
-            for (int e = tid; e < nt * DK; e += kDecodeThreads) sa[e] = expf(sa[e]);
-        } else if (tid < nt) {
-            const float a = expf(sa[tid * DK]);
-            for (int i = 0; i < DK; ++i) sa[tid * DK + i] = a;
+        for (int x = tid; x < nt * DK; x += kTokThreads) {
+            const int tt = x / DK;
+            const float la = gate_per_channel ? sa[x] : sa[tt * DK];
+            rows[x] = make_float4(expf(la), to_f32(sk[x]), to_f32(sq[x]), 0.f);
         }
-        if (warp < nt) {
+        for (int tt = warp; tt < nt; tt += kTokWarps) {
             float acc = 0.f;
-            for (int i = lane; i < DK; i += 32) acc += to_f32(sk[warp * DK + i]) * to_f32(sq[warp * DK + i]);
+            for (int i = lane; i < DK; i += 32) acc += to_f32(sk[tt * DK + i]) * to_f32(sq[tt * DK + i]);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) skq[warp] = acc;
+            if (lane == 0) skq[tt] = acc;
         }
         __syncthreads();
         for (int tt = 0; tt < nt; ++tt) {
-            const int t = t0 + tt, par = t & 1;
-            const float *al = sa + tt * DK;
-            const TIn *kt = sk + tt * DK;
-            const TIn *qt = sq + tt * DK;
-            // S' = Diag(alpha) S and this thread's partial S'^T k, S'^T q
-            uint64_t a0 = f2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+            const float4 *rt = rows + tt * DK;
+            // S' = Diag(alpha) S and this thread's partial S'^T k, S'^T q over its rows
+            uint64_t k01 = f2(0.f, 0.f), k23 = k01, q01 = k01, q23 = k01;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const int i = r * RG + rg;
-                const float ali = al[i], ki = to_f32(kt[i]), qi = to_f32(qt[i]);
-                const uint64_t al2 = f2(ali, ali), k2 = f2(ki, ki), q2 = f2(qi, qi);
-                st[r][0] = mul2(st[r][0], al2);
-                st[r][1] = mul2(st[r][1], al2);
-                a0 = fma2(st[r][0], k2, a0); a1 = fma2(st[r][1], k2, a1);
-                b0 = fma2(st[r][0], q2, b0); b1 = fma2(st[r][1], q2, b1);
+            for (int m = 0; m < RPT; ++m) {
+                const float4 x = rt[rs + NR * m];
+                const uint64_t a2 = f2(x.x, x.x), k2 = f2(x.y, x.y), q2 = f2(x.z, x.z);
+                st[m][0] = mul2(st[m][0], a2);
+                st[m][1] = mul2(st[m][1], a2);
+                k01 = fma2(st[m][0], k2, k01); k23 = fma2(st[m][1], k2, k23);
+                q01 = fma2(st[m][0], q2, q01); q23 = fma2(st[m][1], q2, q23);
             }
-            float4 a, bq;
-            f2_get(a0, a.x, a.y); f2_get(a1, a.z, a.w);
-            f2_get(b0, bq.x, bq.y); f2_get(b1, bq.z, bq.w);
-            float *rk = red + ((size_t)par * 2 + 0) * RG * DV, *rq = red + ((size_t)par * 2 + 1) * RG * DV;
-            reinterpret_cast<float4 *>(rk + rg * DV)[cg] = a;
-            reinterpret_cast<float4 *>(rq + rg * DV)[cg] = bq;
-            __syncthreads();
-            // u = beta (v - S'^T k), o = scale (S'^T q + (k^T q) u), per value column
-            if (tid < DV) {
-                float sk2 = 0.f, sq2 = 0.f;
+            float w[8];
+            f2_get(k01, w[0], w[1]); f2_get(k23, w[2], w[3]);
+            f2_get(q01, w[4], w[5]); f2_get(q23, w[6], w[7]);
+            // sum over the row-set lanes (bits LNC .. 4): the first three steps
+            // halve the vector (k | q, then column pairs, then columns), any
+            // further step adds its partner's copy
 #pragma unroll
-                for (int g = 0; g < RG; ++g) { sk2 += rk[g * DV + tid]; sq2 += rq[g * DV + tid]; }
-                const float u = sb[tt] * (to_f32(sv[tt * DV + tid]) - sk2);
-                su[par * DV + tid] = u;
-                o[tok_index(t) * DV + tid] = from_f32<TIn>(scale * (sq2 + skq[tt] * u));
+            for (int s = 0; s < 5 - LNC; ++s) {
+                const int bit = 16 >> s;
+                if (s < 3) {
+                    const int half = 4 >> s;
+                    const bool up = lane & bit;
+#pragma unroll
+                    for (int e = 0; e < half; ++e) {
+                        const float send = up ? w[e] : w[e + half];
+                        const float keep = up ? w[e + half] : w[e];
+                        w[e] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+                    }
+                } else {
+                    w[0] += __shfl_xor_sync(0xffffffffu, w[0], bit);
+                }
             }
-            __syncthreads();
-            // S = S' + k u^T
-            const float4 u4 = reinterpret_cast<const float4 *>(su + par * DV)[cg];
-            const uint64_t u01 = f2(u4.x, u4.y), u23 = f2(u4.z, u4.w);
+            // u = beta (v - S'^T k) on the k lanes, o = scale (S'^T q + (k^T q) u)
+            // on the q lanes, S = S' + k u^T everywhere
+            const float u = is_q ? 0.f : sb[tt] * (to_f32(sv[tt * DV + c0 + e_own]) - w[0]);
+            const float u_q = __shfl_xor_sync(0xffffffffu, u, 16);
+            if (is_q && primary) so[tt * DV + c0 + e_own] = from_f32<TIn>(scale * (w[0] + skq[tt] * u_q));
+            float u4[4];
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float ki = to_f32(kt[r * RG + rg]);
-                const uint64_t k2 = f2(ki, ki);
-                st[r][0] = fma2(k2, u01, st[r][0]);
-                st[r][1] = fma2(k2, u23, st[r][1]);
+            for (int e = 0; e < 4; ++e) u4[e] = __shfl_sync(0xffffffffu, u, cc + 4 * e);
+            const uint64_t u01 = f2(u4[0], u4[1]), u23 = f2(u4[2], u4[3]);
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) {
+                const float km = rt[rs + NR * m].y;  // reread: keeps the registers for the state
+                const uint64_t k2 = f2(km, km);
+                st[m][0] = fma2(k2, u01, st[m][0]);
+                st[m][1] = fma2(k2, u23, st[m][1]);
             }
         }
-        // every thread is done with this buffer before block b + 2 lands in it
+        // every warp is done with this block: its output rows leave whole, and
+        // its buffer takes block b + 2
         __syncthreads();
+        constexpr int kOG = CPC * (int)sizeof(TIn) / 16;  // 16-byte pieces of this CTA's columns
+        for (int x = tid; x < nt * kOG; x += kTokThreads) {
+            const int tt = x / kOG, r = x % kOG;
+            *reinterpret_cast<uint4 *>(o + tok_index(t0 + tt) * DV + CPC * part + r * (16 / (int)sizeof(TIn))) =
+                reinterpret_cast<const uint4 *>(so + tt * DV + CPC * part)[r];
+        }
         if (b + 2 < nblocks) stage(b + 2);
     }
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
+    for (int m = 0; m < RPT; ++m) {
         float4 x;
-        f2_get(st[r][0], x.x, x.y);
-        f2_get(st[r][1], x.z, x.w);
-        __stcs(reinterpret_cast<float4 *>(Su + (size_t)(r * RG + rg) * DV) + cg, x);
+        f2_get(st[m][0], x.x, x.y);
+        f2_get(st[m][1], x.z, x.w);
+        __stcs(reinterpret_cast<float4 *>(Su + (size_t)(rs + NR * m) * DV + c0), x);
     }
 }
 
@@ -360,7 +392,7 @@ cudaError_t launch_d(const void *q, const void *k, const void *v, const float *l
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::kBytes);
     if (e != cudaSuccess) return e;
-    kern<<<units, kDecodeThreads, L::kBytes, st>>>(
+    kern<<<units * kTokParts, kTokThreads, L::kBytes, st>>>(
         static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v),
         la, beta, S, T, H, gpc, scale, static_cast<TIn *>(o));
     note_launch();

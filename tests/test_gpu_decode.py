@@ -92,8 +92,9 @@ def test_decode_tokens_vs_oracle(T, dtype, d):
 
 
 def test_decode_tokens_equals_chained_steps():
-    """One T-token call and T single-step calls run the same per-token arithmetic
-    on the same fp32 state, so they agree bit for bit."""
+    """One T-token call and T single-step calls apply the same rule to the same
+    fp32 state; only the order of the fp32 sums over the key rows differs (warp
+    shuffles against shared-memory row groups), so they agree to rounding."""
     N, T, H, d = 4, 5, 3, 128
     x, S = _tokens_problem(N, T, H, d, torch.bfloat16, seed=41)
     g = {k: v.cuda() for k, v in x.items() if isinstance(v, torch.Tensor)}
@@ -104,8 +105,8 @@ def test_decode_tokens_equals_chained_steps():
         o2 = kda.kda_decode_step(g["q"][:, t].contiguous(), g["k"][:, t].contiguous(),
                                  g["v"][:, t].contiguous(), g["log_alpha"][:, t].contiguous(),
                                  g["beta"][:, t].contiguous(), S2, scale=x["scale"])
-        assert torch.equal(o1[:, t], o2), t
-    assert torch.equal(S1, S2)
+        assert rel_l2(o1[:, t], o2.double().cpu().numpy()) <= 4e-3, t  # a bf16 rounding step
+    assert rel_l2(S1, S2.double().cpu().numpy()) <= 1e-5
 
 
 def test_decode_tokens_matches_prefill_continuation():
