@@ -288,7 +288,7 @@ BWD_TRAFFIC_PER_TOKEN_HEAD = 53_027
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def bench_backward(steps, warmup, world, rank, dev, T_b=BWD_T):
+def bench_backward(steps, warmup, world, rank, dev, T_b=BWD_T, algo="token"):
     from gated_delta_rule_132_b200 import kda
     P = I.LONG
     devs = f"cuda:{dev}"
@@ -296,18 +296,19 @@ def bench_backward(steps, warmup, world, rank, dev, T_b=BWD_T):
                        device=devs)
     g = torch.Generator(device=devs).manual_seed(P.seed + 7 + 1000 * rank)
     dO = torch.randn(x["v"].shape, generator=g, device=devs).to(P.dtype)
-    ws = torch.empty(int(kda.lib().kda_chunk_bwd_workspace_size(1, T_b, P.H, P.d, P.d, 0, 1)),
-                     dtype=torch.uint8, device=devs)
+    need = kda.lib().kda_chunk_bwd_workspace_size_ex(1, T_b, P.H, P.d, P.d, 0, 1,
+                                                     kda.BWD_ALGOS[algo])
+    ws = torch.empty(int(need), dtype=torch.uint8, device=devs)
     args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], dO)
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
-        kda.kda_chunk_bwd(*args, workspace=ws)
+        kda.kda_chunk_bwd(*args, workspace=ws, algo=algo)
     torch.cuda.synchronize()
     barrier(world)
 
     def step(i, ev):
         ev[0].record(stream)
-        kda.kda_chunk_bwd(*args, workspace=ws)
+        kda.kda_chunk_bwd(*args, workspace=ws, algo=algo)
         ev[1].record(stream)
 
     total_ms, per = time_region(step, steps, stream, marks=2)
@@ -557,6 +558,8 @@ def run_ours(args, world, rank, dev):
             min(args.steps, 5), args.warmup, world, rank, dev)
         bwd = None if args.no_backward else bench_backward(
             min(args.steps, 3), args.warmup, world, rank, dev, args.bwd_tokens)
+        bwd_c = None if args.no_backward else bench_backward(
+            min(args.steps, 3), args.warmup, world, rank, dev, args.bwd_tokens, algo="chunked")
     value = job_throughput(pre["tokens"], pre["ms"], world)
     summ, kernels = prefill_summary(pre, preset, hbm, tc_peak)
 
@@ -670,6 +673,23 @@ def run_ours(args, world, rank, dev):
                          "traffic": BWD_TRAFFIC_PER_TOKEN_HEAD * bwd["token_heads"],
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz",
                          "timed": "whole kda_chunk_bwd call (plan, bwd_kernel, reduction)"}}
+    if bwd_c is not None:
+        tf = bwd_c["token_heads"] * BWD_FLOP_PER_TOKEN_HEAD / (bwd_c["kern_ms"] / 1e3) / 1e12
+        line["backward_chunked"] = {
+            "workload": bwd_c["workload"] + "_backward",
+            "value": round(job_throughput(bwd_c["tokens"], bwd_c["ms"], world), 1),
+            "unit": "tokens/s", "ms_per_step": round(bwd_c["ms"], 3),
+            "steps": min(args.steps, 3), "warmup": args.warmup,
+            "vs_token_walk": round(bwd["ms"] / bwd_c["ms"], 3),
+            "roofline": {"kernel": "chunk-parallel backward (fp32 CUDA cores)", "bound": "alu",
+                         "achieved": round(tf, 3), "peak": round(FP32_PEAK_TFLOPS, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / FP32_PEAK_TFLOPS, 4),
+                         "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz",
+                         "note": "the token walk's algorithmic flops (28 dk dv per token and "
+                                 "head) over the call's time; the chunked form does more",
+                         "timed": "whole kda_chunk_bwd_ex call (plan, record prep, two chunk "
+                                  "walks, two token-gradient kernels)"}}
     line["clocks"] = clocks.summary()
     if not args.no_e2e:
         e = bench_e2e(pre, max(1, args.e2e_steps), torch.cuda.current_stream())

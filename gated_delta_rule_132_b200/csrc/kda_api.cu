@@ -287,6 +287,9 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtyp
 
 }  // extern "C"
 
+// The backward algorithm AUTO stands for: the token walk.
+static bool bwd_chunked(int algo) { return algo == KDA_BWD_CHUNKED; }
+
 static kda_status_t chunk_bwd(const void *q, const void *k, const void *v, kda_dtype_t dt,
                               const float *log_alpha, const float *beta, const float *S0,
                               const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
@@ -294,8 +297,10 @@ static kda_status_t chunk_bwd(const void *q, const void *k, const void *v, kda_d
                               const float *dS_final, float *grad_q, float *grad_k,
                               float *grad_v, float *grad_log_alpha, float *grad_beta,
                               float *grad_S0, void *workspace, size_t workspace_bytes,
-                              int gate_per_channel, void *stream)
+                              int gate_per_channel, int algo, void *stream)
 {
+    if (algo != KDA_BWD_AUTO && algo != KDA_BWD_TOKEN && algo != KDA_BWD_CHUNKED)
+        return KDA_ERR_INVALID_ARG;
     kda::Problem p;
     kda_status_t st = describe(B, T, H, dk, dv, n_seqs, cu_seqlens != nullptr, dt, &p);
     if (st != KDA_OK) return st;
@@ -308,25 +313,37 @@ static kda_status_t chunk_bwd(const void *q, const void *k, const void *v, kda_d
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return KDA_ERR_ALIGNMENT;
     if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_ALIGNMENT;
-    const size_t need = kda::bwd_workspace_layout(p).total;
+    const bool chunked = bwd_chunked(algo);
+    const size_t need = chunked ? kda::cbwd_workspace_bytes(p) : kda::bwd_workspace_layout(p).total;
     if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
     p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.S0 = S0;
     p.cu_seqlens = cu_seqlens; p.scale = scale; p.gate_per_channel = gate_per_channel;
-    const cudaError_t e = kda::launch_backward(p, dO, dS_final, grad_q, grad_k, grad_v,
+    const cudaError_t e =
+        chunked ? kda::launch_backward_chunked(p, dO, dS_final, grad_q, grad_k, grad_v,
                                                grad_log_alpha, grad_beta, grad_S0, workspace,
-                                               static_cast<cudaStream_t>(stream));
+                                               static_cast<cudaStream_t>(stream))
+                : kda::launch_backward(p, dO, dS_final, grad_q, grad_k, grad_v, grad_log_alpha,
+                                       grad_beta, grad_S0, workspace,
+                                       static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 extern "C" {
 
-size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
-                                    kda_dtype_t dt)
+size_t kda_chunk_bwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
+                                       kda_dtype_t dt, int algo)
 {
+    if (algo != KDA_BWD_AUTO && algo != KDA_BWD_TOKEN && algo != KDA_BWD_CHUNKED) return 0;
     kda::Problem p;
     const bool varlen = n_seqs > 0 && B == 1;
     if (describe(B, T, H, dk, dv, n_seqs, varlen, dt, &p) != KDA_OK) return 0;
-    return kda::bwd_workspace_layout(p).total;
+    return bwd_chunked(algo) ? kda::cbwd_workspace_bytes(p) : kda::bwd_workspace_layout(p).total;
+}
+
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
+                                    kda_dtype_t dt)
+{
+    return kda_chunk_bwd_workspace_size_ex(B, T, H, dk, dv, n_seqs, dt, KDA_BWD_AUTO);
 }
 
 #define KDA_BWD_ARGS q, k, v, dt, log_alpha, beta, S0, cu_seqlens, n_seqs, B, T, H, dk, dv, \
@@ -341,7 +358,7 @@ kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v, kda_dtyp
                            float *grad_beta, float *grad_S0, void *workspace,
                            size_t workspace_bytes, void *stream)
 {
-    return chunk_bwd(KDA_BWD_ARGS, 1, stream);
+    return chunk_bwd(KDA_BWD_ARGS, 1, KDA_BWD_AUTO, stream);
 }
 
 kda_status_t kda_gdn_chunk_bwd(const void *q, const void *k, const void *v, kda_dtype_t dt,
@@ -353,7 +370,19 @@ kda_status_t kda_gdn_chunk_bwd(const void *q, const void *k, const void *v, kda_
                                float *grad_S0, void *workspace, size_t workspace_bytes,
                                void *stream)
 {
-    return chunk_bwd(KDA_BWD_ARGS, 0, stream);
+    return chunk_bwd(KDA_BWD_ARGS, 0, KDA_BWD_AUTO, stream);
+}
+
+kda_status_t kda_chunk_bwd_ex(const void *q, const void *k, const void *v, kda_dtype_t dt,
+                              const float *log_alpha, const float *beta, const float *S0,
+                              const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                              int dk, int dv, float scale, const void *dO,
+                              const float *dS_final, float *grad_q, float *grad_k,
+                              float *grad_v, float *grad_log_alpha, float *grad_beta,
+                              float *grad_S0, void *workspace, size_t workspace_bytes,
+                              int gate_per_channel, int algo, void *stream)
+{
+    return chunk_bwd(KDA_BWD_ARGS, gate_per_channel ? 1 : 0, algo, stream);
 }
 
 }  // extern "C"

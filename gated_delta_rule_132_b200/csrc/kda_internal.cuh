@@ -112,6 +112,13 @@ cudaError_t launch_backward(const Problem &p, const void *dO, const float *dS_fi
                             float *gq, float *gk, float *gv, float *gla, float *gbeta,
                             float *gS0, void *workspace, cudaStream_t stream);
 
+// Chunk-parallel backward (fp32 CUDA cores): per-chunk records, a forward and a
+// reverse walk over the chunks, then the token gradients of all chunks at once.
+size_t cbwd_workspace_bytes(const Problem &p);
+cudaError_t launch_backward_chunked(const Problem &p, const void *dO, const float *dS_final,
+                                    float *gq, float *gk, float *gv, float *gla, float *gbeta,
+                                    float *gS0, void *workspace, cudaStream_t stream);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace kda

@@ -76,10 +76,15 @@ def lib() -> ctypes.CDLL:
                                       _vp, _vp]
         L.kda_chunk_bwd_workspace_size.restype = _sz
         L.kda_chunk_bwd_workspace_size.argtypes = [_i] * 7
+        L.kda_chunk_bwd_workspace_size_ex.restype = _sz
+        L.kda_chunk_bwd_workspace_size_ex.argtypes = [_i] * 8
         for fn in ("kda_chunk_bwd", "kda_gdn_chunk_bwd"):
             getattr(L, fn).restype = _i
             getattr(L, fn).argtypes = ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                         _i, _i, _f] + [_vp] * 9 + [_sz, _vp])
+        L.kda_chunk_bwd_ex.restype = _i
+        L.kda_chunk_bwd_ex.argtypes = ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                        _i, _i, _f] + [_vp] * 9 + [_sz, _i, _i, _vp])
         for fn in ("kda_decode_tokens", "kda_gdn_decode_tokens"):
             getattr(L, fn).restype = _i
             getattr(L, fn).argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -280,17 +285,24 @@ def kda_gdn_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, scale=
                         workspace, o, S_final, algo, gate="head").run(stream)
 
 
+BWD_ALGOS = {"auto": 0, "token": 1, "chunked": 2}
+
+
 def kda_chunk_bwd(q, k, v, log_alpha, beta, dO, S0=None, cu_seqlens=None, scale=None,
-                  dS_final=None, want_dS0=True, workspace=None, gate="channel", stream=None):
-    """Backward of the prefill (C: ``kda_chunk_bwd`` / ``kda_gdn_chunk_bwd``): the
-    gradients of <dO, o> + <dS_final, S_final>.
+                  dS_final=None, want_dS0=True, workspace=None, gate="channel", stream=None,
+                  algo="auto"):
+    """Backward of the prefill (C: ``kda_chunk_bwd_ex``): the gradients of
+    <dO, o> + <dS_final, S_final>.
 
     Arguments as :func:`kda_chunk_fwd` (``gate="head"``: log_alpha [B,T,H]), plus
-    dO [B,T,H,dv] in q's dtype and dS_final [N,H,dk,dv] fp32 or None. Returns a dict
-    of fp32 tensors dq, dk, dv, dlog_alpha, dbeta and dS0 (None unless want_dS0).
+    dO [B,T,H,dv] in q's dtype and dS_final [N,H,dk,dv] fp32 or None. ``algo`` is
+    "auto", "token" (token-by-token walk) or "chunked" (chunk-parallel). Returns a
+    dict of fp32 tensors dq, dk, dv, dlog_alpha, dbeta and dS0 (None unless want_dS0).
     """
     if gate not in ("channel", "head"):
         raise ValueError(f"gate must be 'channel' or 'head', not {gate!r}")
+    if algo not in BWD_ALGOS:
+        raise ValueError(f"algo must be one of {sorted(BWD_ALGOS)}, not {algo!r}")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dtype = q.dtype
@@ -318,17 +330,18 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, dO, S0=None, cu_seqlens=None, scale=
          "dbeta": torch.empty((B, T, H), **f32),
          "dS0": torch.empty((N, H, dk, dv), **f32) if want_dS0 else None}
     n_seqs = N if cu_seqlens is not None else 0
-    need = int(lib().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, n_seqs, _dt(q)))
+    need = int(lib().kda_chunk_bwd_workspace_size_ex(B, T, H, dk, dv, n_seqs, _dt(q),
+                                                     BWD_ALGOS[algo]))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    fn = "kda_chunk_bwd" if gate == "channel" else "kda_gdn_chunk_bwd"
-    st = getattr(lib(), fn)(
+    st = lib().kda_chunk_bwd_ex(
         _p(q), _p(k), _p(v), _dt(q), _p(log_alpha), _p(beta), _p(S0), _p(cu_seqlens),
         int(n_seqs), B, T, H, dk, dv, float(scale), _p(dO), _p(dS_final), _p(g["dq"]),
         _p(g["dk"]), _p(g["dv"]), _p(g["dlog_alpha"]), _p(g["dbeta"]), _p(g["dS0"]),
-        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+        _p(workspace), workspace.numel() * workspace.element_size(),
+        1 if gate == "channel" else 0, BWD_ALGOS[algo], _stream(stream))
     if st != 0:
-        raise KdaError(fn, st)
+        raise KdaError("kda_chunk_bwd_ex", st)
     return g
 
 

@@ -325,6 +325,34 @@ kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v,
  */
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_seqs,
                                     kda_dtype_t qkv_dtype);
+/*
+ * Backward algorithms. KDA_BWD_TOKEN walks every sequence token by token (the
+ * states replayed from checkpoints; what kda_chunk_bwd and kda_gdn_chunk_bwd
+ * run, KDA_BWD_AUTO). KDA_BWD_CHUNKED goes through the chunked form of the
+ * rule: per-chunk records (W, U~, e^g q, e^{g_C - g} k, P, e^{g_C}), a forward
+ * and a reverse walk over the chunks (one CTA per sequence, head and 32 value
+ * columns), then the token gradients of all chunks in parallel; fp32 CUDA-core
+ * arithmetic where every exponential is of a non-positive number, so any gate
+ * is safe. Its workspace holds, per (chunk, head) at d = 128, the record
+ * (148 KB), the entry state and chunk-end gradient (64 KB each), U and dU
+ * (32 KB each) and the token-gradient products (115 KB): about 7.1 KB per
+ * token and head.
+ */
+enum { KDA_BWD_AUTO = 0, KDA_BWD_TOKEN = 1, KDA_BWD_CHUNKED = 2 };
+/* Workspace bytes for a backward algorithm (0 on invalid sizes or algo). */
+size_t kda_chunk_bwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
+                                       kda_dtype_t qkv_dtype, int algo);
+/* kda_chunk_bwd (gate_per_channel 1) or kda_gdn_chunk_bwd (0) with an explicit
+ * algorithm; the workspace is kda_chunk_bwd_workspace_size_ex(..., algo) bytes.
+ * An unknown algo returns KDA_ERR_INVALID_ARG before any device work. */
+kda_status_t kda_chunk_bwd_ex(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                              const float *log_alpha, const float *beta, const float *S0,
+                              const int32_t *cu_seqlens, int n_seqs, int B, int T, int H,
+                              int dk, int dv, float scale, const void *dO,
+                              const float *dS_final, float *grad_q, float *grad_k,
+                              float *grad_v, float *grad_log_alpha, float *grad_beta,
+                              float *grad_S0, void *workspace, size_t workspace_bytes,
+                              int gate_per_channel, int algo, void *stream);
 kda_status_t kda_chunk_bwd(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
                            const float *log_alpha, const float *beta, const float *S0,
                            const int32_t *cu_seqlens, int n_seqs, int B, int T, int H, int dk,

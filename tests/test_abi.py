@@ -163,6 +163,39 @@ def test_chunk_bwd_rejects(L, fn, kw, status):
                           a["stream"]) == status
 
 
+@pytest.mark.parametrize("algo,status", [(3, 1), (-1, 1)])
+def test_chunk_bwd_ex_rejects_unknown_algorithm(L, algo, status):
+    assert L.kda_chunk_bwd_ex(_fake(), _fake(), _fake(), 1, _fake(), _fake(), None, None, 0, 1,
+                              64, 2, 128, 128, 0.1, _fake(), None, _fake(), _fake(), _fake(),
+                              _fake(), _fake(), None, _fake(), 1 << 40, 1, algo, None) == status
+
+
+def test_chunk_bwd_ex_rejects_like_the_plain_call(L):
+    """Bad sizes, dtype, alignment and workspace fail on the host for both algorithms."""
+    for algo in (0, 1, 2):
+        base = [_fake(), _fake(), _fake(), 1, _fake(), _fake(), None, None, 0, 1, 64, 2, 128,
+                128, 0.1, _fake(), None, _fake(), _fake(), _fake(), _fake(), _fake(), None,
+                _fake(), 1 << 40, 1, algo, None]
+        bad_dtype = list(base); bad_dtype[3] = 5
+        bad_head = list(base); bad_head[12] = bad_head[13] = 96
+        small_ws = list(base); small_ws[24] = 64
+        misaligned = list(base); misaligned[15] = _fake(0x10002)
+        assert L.kda_chunk_bwd_ex(*bad_dtype) == 2
+        assert L.kda_chunk_bwd_ex(*bad_head) == 2
+        assert L.kda_chunk_bwd_ex(*small_ws) == 4
+        assert L.kda_chunk_bwd_ex(*misaligned) == 3
+
+
+def test_chunk_bwd_workspace_size_ex(L):
+    token = L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 1)
+    chunked = L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 2)
+    assert token == L.kda_chunk_bwd_workspace_size(1, 8192, 32, 128, 128, 0, 1)
+    assert token == L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 0)
+    # chunked: about 7.1 KB per token and head at d = 128
+    assert 6.5e3 * 8192 * 32 < chunked < 7.5e3 * 8192 * 32
+    assert L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 3) == 0
+
+
 def test_chunk_bwd_workspace_size(L):
     a = L.kda_chunk_bwd_workspace_size(1, 4096, 8, 128, 128, 0, 1)
     b = L.kda_chunk_bwd_workspace_size(1, 4097, 8, 128, 128, 0, 1)
