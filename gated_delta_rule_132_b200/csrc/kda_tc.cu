@@ -787,50 +787,59 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
 #pragma unroll
             for (int j = 0; j < 8; ++j) g[e][j] = run[j];
         }
-        *reinterpret_cast<float4 *>(tot + tg * D + c0) = make_float4(run[0], run[1], run[2], run[3]);
-        *reinterpret_cast<float4 *>(tot + tg * D + c0 + 4) = make_float4(run[4], run[5], run[6], run[7]);
+        *reinterpret_cast<float4 *>(tot + tg * D + 4 * oc) = make_float4(run[0], run[1], run[2], run[3]);
+        *reinterpret_cast<float4 *>(tot + tg * D + 64 + 4 * oc) = make_float4(run[4], run[5], run[6], run[7]);
     }
     __syncthreads();
     if (tid < D) {
         // exclusive prefix over the 16 token groups of channel `tid`, plus the
-        // per-channel constants of the factorised exponentials
+        // per-channel constants of the factorised exponentials; rows of tot and
+        // cst keep channel 8 o + 4 u + e at 64 u + 4 o + e, so that the 16
+        // octets of a warp read each half of their 8 channels as one
+        // contiguous 256-byte line
+        const int pos = ((tid >> 2) & 1) * 64 + (tid >> 3) * 4 + (tid & 3);
         float run = 0.f, g15 = 0.f, g31 = 0.f;
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
             if (q == 4) g15 = run;
             if (q == 8) g31 = run;
-            const float v = tot[q * D + tid];
-            tot[q * D + tid] = run;
+            const float v = tot[q * D + pos];
+            tot[q * D + pos] = run;
             run += v;
         }
         const float gC = run;
-        cst[0 * D + tid] = g15;
-        cst[1 * D + tid] = g31;
-        cst[2 * D + tid] = gC;
-        cst[3 * D + tid] = __expf(-g15);
-        cst[4 * D + tid] = __expf(-g31);
-        cst[5 * D + tid] = __expf(g15 - gC);
-        cst[6 * D + tid] = __expf(g31 - gC);
+        cst[0 * D + pos] = g15;
+        cst[1 * D + pos] = g31;
+        cst[2 * D + pos] = gC;
+        cst[3 * D + pos] = __expf(-g15);
+        cst[4 * D + pos] = __expf(-g31);
+        cst[5 * D + pos] = __expf(g15 - gC);
+        cst[6 * D + pos] = __expf(g31 - gC);
         reinterpret_cast<float *>(sm + Prep2Smem::kF)[tid] = __expf(gC - g31);
         reinterpret_cast<float *>(p.rec + ((size_t)c * H + h) * Record::kBytes + Record::kG)[tid] =
             __expf(gC);
     }
     // Multiplicative factors are exact while e^{g} cannot underflow; otherwise
     // take every factor as a direct exponential of its difference.
+    // (cst rows are permuted; threads 0..127 cover every channel either way)
     const bool fast = __syncthreads_and(tid >= D || cst[2 * D + tid] > -80.f);
 
     uint8_t *rec = p.rec + ((size_t)c * H + h) * Record::kBytes;
+    {
+        const float4 lo = *reinterpret_cast<const float4 *>(tot + tg * D + 4 * oc);
+        const float4 hi = *reinterpret_cast<const float4 *>(tot + tg * D + 64 + 4 * oc);
+        const float go[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float go = tot[tg * D + c0 + j];
+        for (int j = 0; j < 8; ++j) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) g[e][j] += go;
+            for (int e = 0; e < 4; ++e) g[e][j] += go[j];
+        }
     }
     bool clamped = false;
     auto cexp = [&](float x) { if (x > 80.f) { clamped = true; x = 80.f; } return __expf(x); };
     auto ld8 = [&](int row, float *a) {  // 8 per-channel constants of this octet
-        const float4 x = *reinterpret_cast<const float4 *>(cst + row * D + c0);
-        const float4 y = *reinterpret_cast<const float4 *>(cst + row * D + c0 + 4);
+        const float4 x = *reinterpret_cast<const float4 *>(cst + row * D + 4 * oc);
+        const float4 y = *reinterpret_cast<const float4 *>(cst + row * D + 64 + 4 * oc);
         a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w; a[4] = y.x; a[5] = y.y; a[6] = y.z; a[7] = y.w;
     };
     const bool first_half = tg < 8;
@@ -850,16 +859,13 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         for (int j = 0; j < 4; ++j) r2[j] = __hmul2(x2[j], f[j]);
         return r;
     };
-    // the per-channel constants this thread needs, once for its 4 tokens:
-    // g_C, and in the fast form the factors of the reference tokens (first
-    // half: e^{-g_15}, e^{g_15 - g_C}, e^{g_31 - g_C}; second half: e^{-g_31},
-    // e^{g_31 - g_C})
-    float cC[8], cx[8], cy[8], cz[8];
+    // g_C of this thread's channels, once for its 4 tokens; the fast form's
+    // reference-token factors (first half: e^{-g_15}, e^{g_15 - g_C},
+    // e^{g_31 - g_C}; second half: e^{-g_31}, e^{g_31 - g_C}) are read from
+    // shared memory per token, which keeps the loop inside the register
+    // budget of two CTAs per SM without spilling
+    float cC[8];
     ld8(2, cC);
-    if (fast) {
-        if (first_half) { ld8(3, cx); ld8(5, cy); ld8(6, cz); }
-        else { ld8(4, cx); ld8(6, cy); }
-    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int r = tg * 4 + e;
@@ -896,6 +902,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         if (first_half) {
             float c0f[8], c1f[8];
             if (fast) {
+                float cx[8], cy[8], cz[8];
+                ld8(3, cx); ld8(5, cy); ld8(6, cz);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     E[j] *= cx[j];            // e^{g_r - g_15}
@@ -919,6 +927,8 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
             *reinterpret_cast<uint4 *>(sm + Prep2Smem::kAop + kb * 16384 + (32 + r) * 128 + sw) = mul4(qe, f2);
         } else {
             if (fast) {
+                float cx[8], cy[8];
+                ld8(4, cx); ld8(6, cy);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     E[j] *= cx[j];            // e^{g_r - g_31}
@@ -1035,16 +1045,24 @@ __global__ void __launch_bounds__(kPrep2Threads, 2) tc_prep2_kernel(const __grid
         uint8_t *tt = sm + Prep2Smem::kTt;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t w[4];
+            // 8 entries of row r as two float4 reads (entries above the
+            // diagonal hold the inverse's scratch and are not selected)
+            const int sb0 = s0 + h2 * 8;
+            const float4 t0 = *reinterpret_cast<const float4 *>(Ts + r * kLd + sb0);
+            const float4 t1 = *reinterpret_cast<const float4 *>(Ts + r * kLd + sb0 + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(sbeta + sb0);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sbeta + sb0 + 4);
+            const float t8[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            const float b8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float v8[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int sa = s0 + h2 * 8 + 2 * e, sb2 = sa + 1;
-                const float va = sa < r ? Ts[r * kLd + sa] : (sa == r ? 1.f : 0.f);
-                const float vb = sb2 < r ? Ts[r * kLd + sb2] : (sb2 == r ? 1.f : 0.f);
-                w[e] = pack_bf16x2(va * sbeta[sa], vb * sbeta[sb2]);
+            for (int e = 0; e < 8; ++e) {
+                const int sa = sb0 + e;
+                v8[e] = (sa < r ? t8[e] : (sa == r ? 1.f : 0.f)) * b8[e];
             }
-            *reinterpret_cast<uint4 *>(tt + tc::sw128(r, (s0 + h2 * 8) * 2)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(tt + tc::sw128(r, sb0 * 2)) =
+                make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
+                           pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
         }
     }
     tc::fence_proxy_async_smem();
