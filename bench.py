@@ -42,7 +42,7 @@ METRIC = ("KDA prefill tokens/s (H=32,d=128) & decode-step state GB/s vs HBM pea
 # dram__bytes_write.sum of one ncu capture of each kernel on the chunked
 # workload, 4096 records per launch); traffic grows in proportion to the
 # records a launch processes. None: no capture of the current kernel yet.
-TRAFFIC_PER_RECORD = {"prepare": 163_216, "carry": 113_586, "gdn_prepare": 128_306}
+TRAFFIC_PER_RECORD = {"prepare": 162_201, "carry": 113_586, "gdn_prepare": 128_265}
 # Algorithmic work of the prefill per token and head at d = 128, chunk 64: bytes
 # the operation must move (q, k, v bf16 in, log_alpha and beta fp32 in, o bf16
 # out; the states are added per sequence) and tensor-core flops of the chunked

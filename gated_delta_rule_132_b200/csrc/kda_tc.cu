@@ -1138,7 +1138,8 @@ struct GdnSmem {
     static constexpr uint32_t kTu = 103424;   // 8192:  T Diag(beta) bf16, K-major rows r
     static constexpr uint32_t kG = 111616;    // fp32 g [64], beta [64]
     static constexpr uint32_t kBar = 112128;  // barriers + tmem slot + flags
-    static constexpr uint32_t kBytes = kBar + 64 + 1024;
+    static constexpr uint32_t kE = kBar + 64; // fp32 e^{g} [64], e^{g_C - g} [64]
+    static constexpr uint32_t kBytes = kE + 512 + 1024;
     // Later tenants (each region is dead by then):
     static constexpr uint32_t kP = kTw + 8192;  // 8192:  P, from the A/P read-out to MMA-NP
     static constexpr uint32_t kKhT = 49152;     // 16384: K^ rows i, after the T images
@@ -1161,6 +1162,8 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
     uint64_t *bar_ld = bar_ap + 4;
     float *sg = reinterpret_cast<float *>(sm + GdnSmem::kG);
     float *sbeta = sg + C;
+    float *seg = reinterpret_cast<float *>(sm + GdnSmem::kE);  // e^{g_t}
+    float *segk = seg + C;                                       // e^{g_C - g_t}
 
     const int c = blockIdx.x, h = blockIdx.y, H = p.H;
     ChunkLoc loc;
@@ -1200,6 +1203,12 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         }
         sg[r1] = run;
         sg[r0] = run - a1;
+        // the exponentials every later step needs, once per token
+        const float gC = __shfl_sync(0xffffffffu, run, 31);
+        seg[r0] = __expf(run - a1);
+        seg[r1] = __expf(run);
+        segk[r0] = __expf(gC - (run - a1));
+        segk[r1] = __expf(gC - run);
     } else if (warp == 2) {
         for (int r = lane; r < C; r += 32) sbeta[r] = r < L ? p.beta[(size_t)(t0 + r) * H + h] : 0.f;
     }
@@ -1292,17 +1301,29 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
         const int r = tid >> 2, s0 = (tid & 3) * 16;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
+            const int sb0 = s0 + h2 * 8;
+            // 8 entries of row r as float4 reads (entries above the diagonal hold
+            // the inverse's scratch and are not selected)
+            const float4 t0 = *reinterpret_cast<const float4 *>(Ts + r * kLd + sb0);
+            const float4 t1 = *reinterpret_cast<const float4 *>(Ts + r * kLd + sb0 + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(sbeta + sb0);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sbeta + sb0 + 4);
+            const float4 e0 = *reinterpret_cast<const float4 *>(seg + sb0);
+            const float4 e1 = *reinterpret_cast<const float4 *>(seg + sb0 + 4);
+            const float t8[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            const float b8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const float e8[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
             uint32_t ww[4], wu[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int sa = s0 + h2 * 8 + 2 * e, sb2 = sa + 1;
-                const float ta = sa < r ? Ts[r * kLd + sa] : (sa == r ? 1.f : 0.f);
-                const float tb = sb2 < r ? Ts[r * kLd + sb2] : (sb2 == r ? 1.f : 0.f);
-                const float ba = sbeta[sa] * ta, bb = sbeta[sb2] * tb;
+                const int sa = sb0 + 2 * e, sb2 = sa + 1;
+                const float ta = sa < r ? t8[2 * e] : (sa == r ? 1.f : 0.f);
+                const float tb = sb2 < r ? t8[2 * e + 1] : (sb2 == r ? 1.f : 0.f);
+                const float ba = b8[2 * e] * ta, bb = b8[2 * e + 1] * tb;
                 wu[e] = pack_bf16x2(ba, bb);
-                ww[e] = pack_bf16x2(ba * __expf(sg[sa]), bb * __expf(sg[sb2]));
+                ww[e] = pack_bf16x2(ba * e8[2 * e], bb * e8[2 * e + 1]);
             }
-            const uint32_t off = tc::sw128(r, (s0 + h2 * 8) * 2);
+            const uint32_t off = tc::sw128(r, sb0 * 2);
             *reinterpret_cast<uint4 *>(sm + GdnSmem::kTw + off) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
             *reinterpret_cast<uint4 *>(sm + GdnSmem::kTu + off) = make_uint4(wu[0], wu[1], wu[2], wu[3]);
         }
@@ -1344,7 +1365,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
             const int t = 8 * cq + e;
             const __nv_bfloat16 x = *reinterpret_cast<const __nv_bfloat16 *>(
                 sm + GdnSmem::kQK + kb * 16384 + tc::sw128((uint32_t)t, ib));
-            kh[e] = __expf(gC - sg[t]) * __bfloat162float(x);
+            kh[e] = segk[t] * __bfloat162float(x);
         }
         *reinterpret_cast<uint4 *>(sm + GdnSmem::kKhT + tc::sw128((uint32_t)i, 16u * (uint32_t)cq)) =
             make_uint4(pack_bf16x2(kh[0], kh[1]), pack_bf16x2(kh[2], kh[3]),
@@ -1370,7 +1391,7 @@ __global__ void __launch_bounds__(kGdnThreads, 2) tc_gdn_prep_kernel(const __gri
     };
     auto qconv = [&](int t, const uint4 &x, float *q8) {
         const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&x);
-        const float et = __expf(sg[t]);
+        const float et = seg[t];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             q8[2 * e] = et * __low2float(x2[e]);
