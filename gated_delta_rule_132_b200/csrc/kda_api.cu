@@ -141,7 +141,7 @@ const char *kda_status_string(kda_status_t s)
     return "unknown status";
 }
 
-int kda_version(void) { return 300; }  // 0.3.0: device status word, launch count
+int kda_version(void) { return 310; }  // 0.3.1: backward algorithm selection
 
 size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int n_seqs,
                                        kda_dtype_t dt, int algo)
