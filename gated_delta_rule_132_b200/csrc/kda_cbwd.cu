@@ -20,6 +20,21 @@ struct DevX {
     __device__ int block() const { return blockIdx.x; }
     __device__ int block_y() const { return blockIdx.y; }
     __device__ void sync() { __syncthreads(); }
+    // 16-byte asynchronous copy global -> shared (both 16-byte aligned), in
+    // this thread's current group
+    __device__ void cp16(void *dst, const void *src)
+    {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                     ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+    }
+    __device__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+    // wait until at most `pending` of this thread's committed groups are in flight
+    __device__ void cp_wait(int pending)
+    {
+        if (pending <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+        else if (pending == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 2;" ::: "memory");
+    }
 };
 
 template <int D, typename TIn>

@@ -88,8 +88,12 @@ template <int D> CB_HD constexpr size_t rec_floats() { return 4 * (size_t)C * D 
 template <int D> CB_HD constexpr size_t scr_floats() { return 3 * (size_t)C * D + C * C + D; }
 
 template <int D> CB_HD constexpr size_t prep_smem() { return sizeof(float) * (3 * C * (D + 4) + C * D + C * C + C); }
-template <int D> CB_HD constexpr size_t fwd_carry_smem() { return sizeof(float) * (2 * C * D + 2 * C * WV + D * WV + D); }
-template <int D> CB_HD constexpr size_t bwd_carry_smem() { return sizeof(float) * (3 * C * D + C * C + 2 * C * WV + D * WV + D); }
+// forward walk: two buffers of one chunk's W, K^, U~ slice and gamma, then U and S
+template <int D> CB_HD constexpr size_t fwd_buf_floats() { return 2 * (size_t)C * D + C * WV + D; }
+template <int D> CB_HD constexpr size_t fwd_carry_smem() { return sizeof(float) * (2 * fwd_buf_floats<D>() + C * WV + D * WV); }
+// reverse walk: two buffers of one chunk's K^, P and gamma, then W, Q~, P^T, dO, dU and G
+template <int D> CB_HD constexpr size_t bwd_buf_floats() { return (size_t)C * D + C * C + D; }
+template <int D> CB_HD constexpr size_t bwd_carry_smem() { return sizeof(float) * (2 * bwd_buf_floats<D>() + 2 * C * D + C * C + 2 * C * WV + D * WV); }
 template <int D> CB_HD constexpr size_t grad_a_smem() { return sizeof(float) * (3 * C * D + 2 * D * (D < 64 ? D : 64)); }
 template <int D> CB_HD constexpr size_t grad_b_smem() { return sizeof(float) * (3 * C * (D + 4) + 2 * C * D + 2 * C * C + C); }
 
@@ -227,32 +231,52 @@ CB_HD void prep(const CbParams &p, X &x, float *smem, float *rec_out)
 // Forward walk over one (sequence, head, 32-column slice): keeps S at every
 // chunk entry and U = Ut - W S. Thread (grp, j) owns column j; it forms U for
 // rows grp + 8 m and updates the state rows 16 grp .. 16 grp + 15, reading
-// the shared row operands (W, K^) as float4.
+// the shared row operands (W, K^) as float4. The next chunk's W, K^, U~
+// slice and gamma arrive by asynchronous copies into the other of two
+// buffers while this chunk computes.
 template <int D, class X>
 CB_HD void fwd_carry(const CbParams &p, X &x, float *smem)
 {
     constexpr int NS = D / WV, NG = NT / WV, RPG = D / NG;  // state rows per group
     static_assert(RPG % 4 == 0 && RPG >= 4, "state rows per thread group");
     constexpr size_t RS = rec_floats<D>();
-    float *sW = smem, *sK = sW + C * D, *sUt = sK + C * D, *sU = sUt + C * WV;
-    float *sS = sU + C * WV, *sG = sS + D * WV;
+    constexpr size_t BUF = fwd_buf_floats<D>();
+    float *sU = smem + 2 * BUF, *sS = sU + C * WV;
     const int H = p.H, bx = x.block();
     const int j0 = (bx % NS) * WV, h = (bx / NS) % H, n = p.order[bx / (NS * H)];
     const int tid = x.tid(), j = tid % WV, grp = tid / WV, i0 = grp * RPG;
     const size_t sbase = ((size_t)n * H + h) * D * D;
-    for (int i = i0; i < i0 + RPG; ++i) sS[i * WV + j] = p.S0 ? p.S0[sbase + (size_t)i * D + j0 + j] : 0.f;
     const int c0 = p.chunk_off[n], nc = p.chunk_off[n + 1] - c0;
+    // chunk lc's operands into buffer b, as one group of 16-byte copies
+    auto fetch = [&](int lc, int b) {
+        const float *w = p.rec + ((size_t)(c0 + lc) * H + h) * RS;
+        float *bW = smem + b * BUF, *bK = bW + C * D, *bUt = bK + C * D, *bG = bUt + C * WV;
+        for (int i = tid; i < C * D / 4; i += NT) {
+            x.cp16(bW + 4 * i, w + 4 * i);
+            x.cp16(bK + 4 * i, w + 3 * C * D + 4 * i);
+        }
+        for (int i = tid; i < C * WV / 4; i += NT) {
+            const int r = i / (WV / 4), q4 = i % (WV / 4);
+            x.cp16(bUt + r * WV + 4 * q4, w + C * D + (size_t)r * D + j0 + 4 * q4);
+        }
+        for (int i = tid; i < D / 4; i += NT) x.cp16(bG + 4 * i, w + 4 * C * D + C * C + 4 * i);
+        x.cp_commit();
+    };
+    for (int i = i0; i < i0 + RPG; ++i) sS[i * WV + j] = p.S0 ? p.S0[sbase + (size_t)i * D + j0 + j] : 0.f;
+    if (nc > 0) fetch(0, 0);
     for (int lc = 0; lc < nc; ++lc) {
+        const int b = lc & 1;
         const size_t ch = (size_t)(c0 + lc) * H + h;
-        const float *w = p.rec + ch * RS;
+        const float *sW = smem + b * BUF, *sK = sW + C * D, *sUt = sK + C * D, *sG = sUt + C * WV;
         float *Sst = p.Sst + ch * D * D, *Ust = p.Ust + ch * C * D;
         for (int i = i0; i < i0 + RPG; ++i) Sst[(size_t)i * D + j0 + j] = sS[i * WV + j];
-        x.sync();  // the previous chunk is done with the buffers
-        copy4<NT>(sW, w, C * D, tid);
-        copy4<NT>(sK, w + 3 * C * D, C * D, tid);
-        for (int idx = tid; idx < C * WV; idx += NT)
-            sUt[idx] = w[C * D + (idx / WV) * D + j0 + idx % WV];
-        for (int i = tid; i < D; i += NT) sG[i] = w[4 * C * D + C * C + i];
+        x.sync();  // the previous chunk is done with the other buffer, U and S
+        if (lc + 1 < nc) {
+            fetch(lc + 1, b ^ 1);
+            x.cp_wait(1);  // this chunk's group has landed; the next one may still fly
+        } else {
+            x.cp_wait(0);
+        }
         x.sync();
         {
             float acc[C / NG];
@@ -293,14 +317,21 @@ CB_HD void fwd_carry(const CbParams &p, X &x, float *smem)
 // Reverse walk over one (sequence, head, 32-column slice): keeps G (the gradient
 // at each chunk's end) and dU, and returns the slice of dS0. Same thread layout
 // as the forward walk; Pm is kept transposed so its column reads are float4.
+// The operands of the dU step (K^, P, gamma) come one chunk ahead into the
+// other of two buffers, and dO one chunk ahead into registers; W and Q~,
+// needed only by the G step, are copied at the start of the chunk and land
+// while the dU step runs.
 template <int D, typename TIn, class X>
 CB_HD void bwd_carry(const CbParams &p, X &x, float *smem)
 {
     constexpr int NS = D / WV, NG = NT / WV, RPG = D / NG;
     static_assert(RPG % 4 == 0 && RPG >= 4, "state rows per thread group");
     constexpr size_t RS = rec_floats<D>();
-    float *sW = smem, *sQ = sW + C * D, *sK = sQ + C * D, *sPt = sK + C * D;
-    float *sdO = sPt + C * C, *sdU = sdO + C * WV, *sG = sdU + C * WV, *sgam = sG + D * WV;
+    constexpr size_t BUF = bwd_buf_floats<D>();
+    constexpr int DOPT = C * WV / NT;  // dO values per thread
+    static_assert(C * WV % NT == 0, "dO slice per thread");
+    float *sW = smem + 2 * BUF, *sQ = sW + C * D, *sPt = sQ + C * D;
+    float *sdO = sPt + C * C, *sdU = sdO + C * WV, *sG = sdU + C * WV;
     const int H = p.H, bx = x.block();
     const int j0 = (bx % NS) * WV, h = (bx / NS) % H, n = p.order[bx / (NS * H)];
     const int tid = x.tid(), j = tid % WV, grp = tid / WV, i0 = grp * RPG;
@@ -311,22 +342,49 @@ CB_HD void bwd_carry(const CbParams &p, X &x, float *smem)
         sG[i * WV + j] = p.dS_final ? p.dS_final[sbase + (size_t)i * D + j0 + j] : 0.f;
     const int ts = p.seq_start[n], te = p.seq_start[n + 1];
     const int c0 = p.chunk_off[n], nc = p.chunk_off[n + 1] - c0;
-    for (int lc = nc - 1; lc >= 0; --lc) {
-        const size_t ch = (size_t)(c0 + lc) * H + h;
-        const float *w = p.rec + ch * RS;
+    auto rec_of = [&](int lc) { return p.rec + ((size_t)(c0 + lc) * H + h) * RS; };
+    // chunk lc's K^, P and gamma into buffer b, as one group
+    auto fetch = [&](int lc, int b) {
+        const float *w = rec_of(lc);
+        float *bK = smem + b * BUF, *bP = bK + C * D, *bg = bP + C * C;
+        for (int i = tid; i < C * D / 4; i += NT) x.cp16(bK + 4 * i, w + 3 * C * D + 4 * i);
+        for (int i = tid; i < C * C / 4; i += NT) x.cp16(bP + 4 * i, w + 4 * C * D + 4 * i);
+        for (int i = tid; i < D / 4; i += NT) x.cp16(bg + 4 * i, w + 4 * C * D + C * C + 4 * i);
+        x.cp_commit();
+    };
+    // chunk lc's dO slice (zero past the sequence's end) into registers
+    float dOr[DOPT];
+    auto load_dO = [&](int lc) {
         const int t0 = ts + lc * C, L = te - t0 < C ? te - t0 : C;
+        for (int e = 0; e < DOPT; ++e) {
+            const int idx = tid + NT * e, r = idx / WV, jj = idx % WV;
+            dOr[e] = r < L ? cvt(dO[((size_t)(t0 + r) * H + h) * D + j0 + jj]) : 0.f;
+        }
+    };
+    if (nc > 0) {
+        fetch(nc - 1, (nc - 1) & 1);
+        load_dO(nc - 1);
+    }
+    for (int lc = nc - 1; lc >= 0; --lc) {
+        const int b = lc & 1;
+        const size_t ch = (size_t)(c0 + lc) * H + h;
+        const float *w = rec_of(lc);
+        const float *sK = smem + b * BUF, *sP = sK + C * D, *sgam = sP + C * C;
         float *dSst = p.dSst + ch * D * D, *dUst = p.dUst + ch * C * D;
         for (int i = i0; i < i0 + RPG; ++i) dSst[(size_t)i * D + j0 + j] = sG[i * WV + j];
-        x.sync();
-        copy4<NT>(sW, w, C * D, tid);
-        copy4<NT>(sQ, w + 2 * C * D, C * D, tid);
-        copy4<NT>(sK, w + 3 * C * D, C * D, tid);
-        for (int idx = tid; idx < C * C; idx += NT) sPt[(idx % C) * C + idx / C] = w[4 * C * D + idx];
-        for (int i = tid; i < D; i += NT) sgam[i] = w[4 * C * D + C * C + i];
-        for (int idx = tid; idx < C * WV; idx += NT) {
-            const int r = idx / WV, jj = idx % WV;
-            sdO[idx] = r < L ? cvt(dO[((size_t)(t0 + r) * H + h) * D + j0 + jj]) : 0.f;
+        x.sync();  // the previous chunk is done with W, Q~, P^T, dO, dU and the other buffer
+        for (int i = tid; i < C * D / 4; i += NT) {
+            x.cp16(sW + 4 * i, w + 4 * i);
+            x.cp16(sQ + 4 * i, w + 2 * C * D + 4 * i);
         }
+        x.cp_commit();
+        if (lc > 0) fetch(lc - 1, b ^ 1);
+        else x.cp_commit();  // an empty group keeps the count of groups in flight
+        x.cp_wait(2);        // this chunk's K^, P and gamma have landed
+        for (int e = 0; e < DOPT; ++e) sdO[tid + NT * e] = dOr[e];
+        x.sync();
+        for (int idx = tid; idx < C * C; idx += NT) sPt[(idx % C) * C + idx / C] = sP[idx];
+        if (lc > 0) load_dO(lc - 1);
         x.sync();
         {
             float acc[C / NG], pa[C / NG];
@@ -357,6 +415,7 @@ CB_HD void bwd_carry(const CbParams &p, X &x, float *smem)
                 dUst[(size_t)r * D + j0 + j] = du;
             }
         }
+        x.cp_wait(1);  // W and Q~ have landed (the next chunk's group may still fly)
         x.sync();
         {
             float qd[RPG], wd[RPG];
@@ -379,6 +438,7 @@ CB_HD void bwd_carry(const CbParams &p, X &x, float *smem)
             }
         }
     }
+    x.cp_wait(0);
     if (p.gS0)
         for (int i = i0; i < i0 + RPG; ++i) p.gS0[sbase + (size_t)i * D + j0 + j] = sG[i * WV + j];
 }

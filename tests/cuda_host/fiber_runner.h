@@ -9,6 +9,8 @@
 
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
+#include <utility>
 #include <functional>
 #include <vector>
 
@@ -17,12 +19,31 @@ struct FiberRunner;
 struct HostX {
     int t, bx, by;
     FiberRunner *R;
+    // asynchronous 16-byte copies of this thread: committed groups, oldest
+    // first, and the group being filled. A copy takes effect only when a wait
+    // retires its group, so reading a buffer before waiting sees the old data.
+    std::vector<std::vector<std::pair<void *, const void *>>> groups = {};
+    std::vector<std::pair<void *, const void *>> open = {};
     int tid() const { return t; }
     int block() const { return bx; }
     int block_y() const { return by; }
     void sync();
     void syncwarp();
     float shfl_xor(float v, int lane_mask);
+    void cp16(void *dst, const void *src) { open.push_back({dst, src}); }
+    void cp_commit()
+    {
+        groups.push_back(open);
+        open.clear();
+    }
+    // retire all but the newest `pending` committed groups
+    void cp_wait(int pending)
+    {
+        while ((int)groups.size() > pending) {
+            for (auto &c : groups.front()) std::memcpy(c.first, c.second, 16);
+            groups.erase(groups.begin());
+        }
+    }
 };
 
 struct FiberRunner {
