@@ -287,8 +287,9 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtyp
 
 }  // extern "C"
 
-// The backward algorithm AUTO stands for: the token walk.
-static bool bwd_chunked(int algo) { return algo == KDA_BWD_CHUNKED; }
+// The backward algorithm AUTO stands for: the chunk-parallel form (faster than
+// the token walk on long sequences, with a smaller workspace).
+static bool bwd_chunked(int algo) { return algo != KDA_BWD_TOKEN; }
 
 static kda_status_t chunk_bwd(const void *q, const void *k, const void *v, kda_dtype_t dt,
                               const float *log_alpha, const float *beta, const float *S0,

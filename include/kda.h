@@ -302,23 +302,24 @@ kda_status_t kda_gdn_decode_tokens(const void *q, const void *k, const void *v,
 
 /*
  * Backward of the prefill (for training; the pages state only the forward rule,
- * so this is the rule's derivative, taken token by token in reverse order):
- * the gradients of
+ * so this is the rule's derivative): the gradients of
  *     L = <dO, o> + <dS_final, S_final>
  * with respect to q, k, v, log_alpha, beta and S0, for the arguments of
  * kda_chunk_fwd (same layouts, sequences and scale). Computed in fp32 on CUDA
- * cores for every supported head size; the states are replayed from
- * checkpoints kept every 32 tokens in the workspace. The workspace also holds
- * per-slice partial gradients (dk / 32 slices of 32 value columns), which a
- * second kernel adds in a fixed order, so results are deterministic. At
- * d = 128 it takes about 8.2 KB per token and head plus 2.2 MB per (sequence,
- * head), e.g. 2.2 GB for B = 1, H = 32, T = 8192.
+ * cores for every supported head size, by the chunk-parallel form below
+ * (KDA_BWD_AUTO; results are deterministic). The token walk (KDA_BWD_TOKEN,
+ * through kda_chunk_bwd_ex) replays the states from checkpoints kept every 32
+ * tokens and adds per-slice partial gradients (dk / 32 slices of 32 value
+ * columns) in a fixed order; at d = 128 its workspace is about 8.2 KB per
+ * token and head plus 2.2 MB per (sequence, head), e.g. 2.2 GB for B = 1,
+ * H = 32, T = 8192.
  *   dO              qkv_dtype [B, T, H, dv]
  *   dS_final        fp32 [N, H, dk, dv] or NULL (zero)
  *   grad_q, grad_k  fp32 [B, T, H, dk]       grad_v     fp32 [B, T, H, dv]
  *   grad_log_alpha  fp32 [B, T, H, dk]       grad_beta  fp32 [B, T, H]
  *   grad_S0         fp32 [N, H, dk, dv] or NULL (not returned)
- * Workspace: kda_chunk_bwd_workspace_size bytes. Errors as kda_chunk_fwd_ex.
+ * Workspace: kda_chunk_bwd_workspace_size bytes (that of KDA_BWD_AUTO). Errors as
+ * kda_chunk_fwd_ex.
  * Tokens outside every sequence (cu_seqlens ending before B*T) are not written.
  * kda_gdn_chunk_bwd: the same for one gate per token and head (log_alpha and
  * grad_log_alpha fp32 [B, T, H]).
@@ -327,9 +328,9 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int n_s
                                     kda_dtype_t qkv_dtype);
 /*
  * Backward algorithms. KDA_BWD_TOKEN walks every sequence token by token (the
- * states replayed from checkpoints; what kda_chunk_bwd and kda_gdn_chunk_bwd
- * run, KDA_BWD_AUTO). KDA_BWD_CHUNKED goes through the chunked form of the
- * rule: per-chunk records (W, U~, e^g q, e^{g_C - g} k, P, e^{g_C}), a forward
+ * states replayed from checkpoints). KDA_BWD_CHUNKED goes through the chunked
+ * form of the rule (what kda_chunk_bwd and kda_gdn_chunk_bwd run, and
+ * KDA_BWD_AUTO): per-chunk records (W, U~, e^g q, e^{g_C - g} k, P, e^{g_C}), a forward
  * and a reverse walk over the chunks (one CTA per sequence, head and 32 value
  * columns), then the token gradients of all chunks in parallel; fp32 CUDA-core
  * arithmetic where every exponential is of a non-positive number, so any gate

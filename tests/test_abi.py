@@ -189,8 +189,10 @@ def test_chunk_bwd_ex_rejects_like_the_plain_call(L):
 def test_chunk_bwd_workspace_size_ex(L):
     token = L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 1)
     chunked = L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 2)
-    assert token == L.kda_chunk_bwd_workspace_size(1, 8192, 32, 128, 128, 0, 1)
-    assert token == L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 0)
+    # AUTO is the chunk-parallel form, also for the plain size query
+    assert chunked == L.kda_chunk_bwd_workspace_size(1, 8192, 32, 128, 128, 0, 1)
+    assert chunked == L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 0)
+    assert token > chunked
     # chunked: about 7.1 KB per token and head at d = 128
     assert 6.5e3 * 8192 * 32 < chunked < 7.5e3 * 8192 * 32
     assert L.kda_chunk_bwd_workspace_size_ex(1, 8192, 32, 128, 128, 0, 1, 3) == 0
