@@ -274,9 +274,11 @@ def bench_gdn(pre, steps, warmup, world):
                 carry_ms=statistics.mean(p[1] for p in per), in_bytes=in_b)
 
 
-# The backward (kda_chunk_bwd) on the long workload's shape cut to its first 8192
-# tokens: fp32 CUDA-core arithmetic, ~28 dk*dv flop per token and head (two
-# forward replays and the reverse step).
+# The backward (kda_chunk_bwd_ex, both algorithms: the token walk under the key
+# "backward", the chunk-parallel default under "backward_chunked") on the long
+# workload's shape cut to its first 8192 tokens: fp32 CUDA-core arithmetic; the
+# token walk does ~28 dk*dv flop per token and head (two forward replays and the
+# reverse step), which both keys count as the algorithmic work.
 BWD_T = 8192
 BWD_FLOP_PER_TOKEN_HEAD = 28 * 128 * 128
 # DRAM bytes (read + write) of bwd_kernel per token and head: one ncu capture at
@@ -692,7 +694,8 @@ def run_ours(args, world, rank, dev):
                          "unit": "TFLOP/s", "frac": round(tf / FP32_PEAK_TFLOPS, 4),
                          "traffic": BWD_TRAFFIC_PER_TOKEN_HEAD * bwd["token_heads"],
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz",
-                         "timed": "whole kda_chunk_bwd call (plan, bwd_kernel, reduction)"}}
+                         "timed": "whole kda_chunk_bwd_ex call with the token walk (plan, "
+                                  "bwd_kernel, reduction)"}}
     if bwd_c is not None:
         tf = bwd_c["token_heads"] * BWD_FLOP_PER_TOKEN_HEAD / (bwd_c["kern_ms"] / 1e3) / 1e12
         line["backward_chunked"] = {
