@@ -136,9 +136,9 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 // (barrier); then every warp runs the block's tokens on its own columns; o goes
 // to a staging tile and leaves as full row pieces after a last barrier, when the
 // buffer is also free for block b + 2. The value columns of a head never mix,
-// so a head's 8 column slices of dv / 8 are spread over kTokParts CTAs of
-// 8 / kTokParts warps each (smaller CTAs overlap one another's loads and
-// arithmetic better).
+// so a head's 8 column slices of dv / 8 may be spread over kTokParts CTAs of
+// 8 / kTokParts warps each; one CTA per head measured fastest (2 and 4 CTAs of
+// fewer warps were slower at every T tried).
 constexpr int kTokBlock = 8;
 constexpr int kTokParts = 1;                      // CTAs per (sequence, head)
 constexpr int kTokWarps = 8 / kTokParts;          // warps per CTA
